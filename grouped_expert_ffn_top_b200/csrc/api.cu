@@ -1,0 +1,287 @@
+// The C ABI (include/moe.h): argument checks, workspace carving and launches.
+// Every check runs before anything is launched, so a rejected call changes
+// nothing on the device.
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return MOE_OK;
+  return fail(MOE_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool dtype_ok(int dtype) { return dtype == MOE_F32 || dtype == MOE_BF16; }
+size_t elem_bytes(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+size_t align256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Common checks of the row-wise passes (permute / combine and their backward).
+int check_rows(const char* fn, int dtype, int64_t T, int d, int k) {
+  if (!dtype_ok(dtype)) return fail(MOE_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, dtype);
+  if (T < 0 || d < 1 || k < 1) return fail(MOE_ERR_INVALID_ARG, "%s: T=%lld d=%d k=%d", fn,
+                                           static_cast<long long>(T), d, k);
+  if (k > 32) return fail(MOE_ERR_UNSUPPORTED, "%s: k=%d > 32", fn, k);
+  if (d % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "%s: d=%d is not a multiple of 8", fn, d);
+  if (T * k >= (int64_t(1) << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "%s: T*k=%lld rows exceed int32", fn,
+                static_cast<long long>(T * k));
+  return MOE_OK;
+}
+
+int check_ffn(const char* fn, int dtype, int64_t rows, int E, int d, int f) {
+  if (!dtype_ok(dtype)) return fail(MOE_ERR_UNSUPPORTED, "%s: unknown dtype %d", fn, dtype);
+  if (rows < 0 || E < 1 || d < 1 || f < 1)
+    return fail(MOE_ERR_INVALID_ARG, "%s: rows=%lld E=%d d=%d f=%d", fn,
+                static_cast<long long>(rows), E, d, f);
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "%s: E=%d > %d", fn, E, MOE_MAX_EXPERTS);
+  if (rows >= (int64_t(1) << 31)) return fail(MOE_ERR_UNSUPPORTED, "%s: rows exceed int32", fn);
+  const int q = dtype == MOE_BF16 ? 64 : 4;
+  if (d % q != 0 || f % q != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "%s: d=%d and f=%d must be multiples of %d for this dtype",
+                fn, d, f, q);
+  if (static_cast<int64_t>(E) * (d > f ? d : f) >= (int64_t(1) << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "%s: E*max(d,f) exceeds int32", fn);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error(void) { return g_msg; }
+
+int moe_version(void) { return 1; }
+
+int moe_get_error(void* ws, cudaStream_t stream) {
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "moe_get_error: null workspace");
+  unsigned h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(unsigned), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(unsigned), stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_status(e, "moe_get_error");
+  return static_cast<int>(h & 0x7fffffffu);
+}
+
+// ------------------------------------------------------------------ routing
+
+int moe_router_logits(const void* x, const void* Wr, const float* b, int dtype, int64_t T, int d,
+                      int E, float* logits, cudaStream_t stream) {
+  if (!dtype_ok(dtype)) return fail(MOE_ERR_UNSUPPORTED, "moe_router_logits: dtype %d", dtype);
+  if (T < 0 || d < 1 || E < 1) return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: sizes");
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_router_logits: E=%d", E);
+  if (d % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "moe_router_logits: d=%d not a multiple of 8", d);
+  if (T == 0) return MOE_OK;
+  if (!x || !Wr || !logits) return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: null pointer");
+  return cuda_status(moe::launch_router_logits(x, Wr, b, dtype, T, d, E, logits, stream),
+                     "moe_router_logits");
+}
+
+size_t moe_route_workspace_bytes(int64_t T, int E) {
+  if (T < 0 || E < 1) return 0;
+  const int64_t nb = (T + moe::kRouteTokensPerBlock - 1) / moe::kRouteTokensPerBlock;
+  return moe::kWsHeader + 2 * align256(sizeof(int32_t) * static_cast<size_t>(nb) * E);
+}
+
+int moe_route(const float* logits, int64_t T, int E, int k, int ep_groups, int32_t* topk_idx,
+              float* topk_w, int32_t* expert_counts, int64_t* expert_offsets,
+              int32_t* group_counts, int64_t* group_offsets, int32_t* row_of_pair,
+              int32_t* pair_of_row, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E || ep_groups < 1)
+    return fail(MOE_ERR_INVALID_ARG, "moe_route: T=%lld E=%d k=%d ep_groups=%d",
+                static_cast<long long>(T), E, k, ep_groups);
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_route: E=%d > %d", E, MOE_MAX_EXPERTS);
+  if (k > 32) return fail(MOE_ERR_UNSUPPORTED, "moe_route: k=%d > 32", k);
+  if (E % ep_groups != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_route: E=%d is not divisible by ep_groups=%d", E,
+                ep_groups);
+  if (T * k >= (int64_t(1) << 31)) return fail(MOE_ERR_UNSUPPORTED, "moe_route: T*k exceeds int32");
+  if (T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_w || !expert_counts || !expert_offsets || !group_counts ||
+      !group_offsets || !row_of_pair || !pair_of_row || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_route: null pointer");
+  if (ws_bytes < moe_route_workspace_bytes(T, E) || !aligned16(ws))
+    return fail(MOE_ERR_WORKSPACE, "moe_route: workspace needs %zu bytes (got %zu), 16-aligned",
+                moe_route_workspace_bytes(T, E), ws_bytes);
+  const int64_t nb = (T + moe::kRouteTokensPerBlock - 1) / moe::kRouteTokensPerBlock;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  unsigned* err = reinterpret_cast<unsigned*>(base);
+  int32_t* block_counts = reinterpret_cast<int32_t*>(base + moe::kWsHeader);
+  int32_t* block_base = reinterpret_cast<int32_t*>(
+      base + moe::kWsHeader + align256(sizeof(int32_t) * static_cast<size_t>(nb) * E));
+  if (E > 768) {
+    cudaError_t e = moe::route_set_smem_limits();
+    if (e != cudaSuccess) return cuda_status(e, "moe_route");
+  }
+  return cuda_status(moe::launch_route(logits, T, E, k, ep_groups, topk_idx, topk_w, expert_counts,
+                                       expert_offsets, group_counts, group_offsets, row_of_pair,
+                                       pair_of_row, block_counts, block_base, err, stream),
+                     "moe_route");
+}
+
+int moe_route_bwd(const float* dg, const float* topk_w, const int32_t* topk_idx, int64_t T, int E,
+                  int k, float* dlogits, cudaStream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "moe_route_bwd: sizes");
+  if (k > 32) return fail(MOE_ERR_UNSUPPORTED, "moe_route_bwd: k=%d > 32", k);
+  if (T == 0) return MOE_OK;
+  if (!dg || !topk_w || !topk_idx || !dlogits)
+    return fail(MOE_ERR_INVALID_ARG, "moe_route_bwd: null pointer");
+  return cuda_status(moe::launch_route_bwd(dg, topk_w, topk_idx, T, E, k, dlogits, stream),
+                     "moe_route_bwd");
+}
+
+// ----------------------------------------------------------------- dispatch
+
+int moe_permute(const void* x, int dtype, int64_t T, int d, int k, const int32_t* row_of_pair,
+                void* xp, cudaStream_t stream) {
+  int rc = check_rows("moe_permute", dtype, T, d, k);
+  if (rc != MOE_OK) return rc;
+  if (T == 0) return MOE_OK;
+  if (!x || !row_of_pair || !xp) return fail(MOE_ERR_INVALID_ARG, "moe_permute: null pointer");
+  if (!aligned16(x) || !aligned16(xp)) return fail(MOE_ERR_INVALID_ARG, "moe_permute: 16-byte alignment");
+  return cuda_status(moe::launch_permute(x, dtype, T, d, k, row_of_pair, xp, stream), "moe_permute");
+}
+
+int moe_unpermute_combine(const void* yp, const float* topk_w, const int32_t* row_of_pair,
+                          int dtype, int64_t T, int d, int k, void* Y, cudaStream_t stream) {
+  int rc = check_rows("moe_unpermute_combine", dtype, T, d, k);
+  if (rc != MOE_OK) return rc;
+  if (T == 0) return MOE_OK;
+  if (!yp || !topk_w || !row_of_pair || !Y)
+    return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine: null pointer");
+  if (!aligned16(yp) || !aligned16(Y))
+    return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine: 16-byte alignment");
+  return cuda_status(moe::launch_combine(yp, topk_w, row_of_pair, dtype, T, d, k, Y, stream),
+                     "moe_unpermute_combine");
+}
+
+int moe_unpermute_combine_bwd(const void* dY, const void* yp, const float* topk_w,
+                              const int32_t* row_of_pair, int dtype, int64_t T, int d, int k,
+                              void* dyp, float* dg, cudaStream_t stream) {
+  int rc = check_rows("moe_unpermute_combine_bwd", dtype, T, d, k);
+  if (rc != MOE_OK) return rc;
+  if (T == 0) return MOE_OK;
+  if (!dY || !yp || !topk_w || !row_of_pair || !dyp || !dg)
+    return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine_bwd: null pointer");
+  if (!aligned16(dY) || !aligned16(yp) || !aligned16(dyp))
+    return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine_bwd: 16-byte alignment");
+  return cuda_status(
+      moe::launch_combine_bwd(dY, yp, topk_w, row_of_pair, dtype, T, d, k, dyp, dg, stream),
+      "moe_unpermute_combine_bwd");
+}
+
+int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dlogits,
+                    const void* Wr, const int32_t* topk_idx, int dtype, int64_t T, int d, int E,
+                    int k, void* dX, cudaStream_t stream) {
+  int rc = check_rows("moe_permute_bwd", dtype, T, d, k);
+  if (rc != MOE_OK) return rc;
+  if (E < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "moe_permute_bwd: E=%d k=%d", E, k);
+  if (T == 0) return MOE_OK;
+  if (!dxp || !row_of_pair || !dX || (dlogits && (!Wr || !topk_idx)))
+    return fail(MOE_ERR_INVALID_ARG, "moe_permute_bwd: null pointer");
+  if (!aligned16(dxp) || !aligned16(dX) || (dlogits && !aligned16(Wr)))
+    return fail(MOE_ERR_INVALID_ARG, "moe_permute_bwd: 16-byte alignment");
+  return cuda_status(moe::launch_permute_bwd(dxp, row_of_pair, dlogits, Wr, topk_idx, dtype, T, d,
+                                             E, k, dX, stream),
+                     "moe_permute_bwd");
+}
+
+size_t moe_router_bwd_workspace_bytes(int64_t T, int d, int E) {
+  if (T < 0 || d < 1 || E < 1) return 0;
+  const int S = moe::router_bwd_splits(T, d, E);
+  return moe::kWsHeader + align256(sizeof(float) * static_cast<size_t>(S) * E * (d + 1));
+}
+
+int moe_router_bwd(const void* x, const float* dlogits, int dtype, int64_t T, int d, int E,
+                   float* dWr, float* db, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!dtype_ok(dtype)) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd: dtype %d", dtype);
+  if (T < 0 || d < 1 || E < 1) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: sizes");
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd: E=%d", E);
+  if (T == 0) return MOE_OK;
+  if (!x || !dlogits || !dWr || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: null pointer");
+  if (ws_bytes < moe_router_bwd_workspace_bytes(T, d, E) || !aligned16(ws))
+    return fail(MOE_ERR_WORKSPACE, "moe_router_bwd: workspace needs %zu bytes",
+                moe_router_bwd_workspace_bytes(T, d, E));
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + moe::kWsHeader);
+  return cuda_status(moe::launch_router_bwd(x, dlogits, dtype, T, d, E, dWr, db, partial, stream),
+                     "moe_router_bwd");
+}
+
+// ------------------------------------------------------------ grouped FFN
+
+size_t moe_grouped_ffn_fwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype) {
+  (void)rows; (void)E; (void)d; (void)f; (void)dtype;
+  return moe::kWsHeader;
+}
+
+int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const void* Wd, int dtype,
+                        const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
+                        void* h1, void* h2, void* a, void* yp, void* ws, size_t ws_bytes,
+                        cudaStream_t stream) {
+  int rc = check_ffn("moe_grouped_ffn_fwd", dtype, rows, E, d, f);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!xp || !Wg || !Wu || !Wd || !expert_offsets || !h1 || !h2 || !a || !yp || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd: null pointer");
+  const void* ptrs[] = {xp, Wg, Wu, Wd, h1, h2, a, yp, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd: 16-byte alignment");
+  if (ws_bytes < moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_fwd: workspace too small");
+  moe::FfnFwdArgs args{xp, Wg, Wu, Wd, expert_offsets, rows, E, d, f, h1, h2, a, yp,
+                       static_cast<unsigned*>(ws)};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_fwd_bf16(args, stream)
+                                    : moe::launch_ffn_fwd_f32(args, stream);
+  return cuda_status(e, "moe_grouped_ffn_fwd");
+}
+
+size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype) {
+  (void)E; (void)d;
+  if (rows < 0 || f < 1 || !dtype_ok(dtype)) return 0;
+  const size_t h = align256(static_cast<size_t>(rows) * f * elem_bytes(dtype));
+  return moe::kWsHeader + 2 * h;
+}
+
+int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,
+                        const void* h1, const void* h2, const void* a, const void* dyp, int dtype,
+                        const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
+                        void* dxp, float* dWg, float* dWu, float* dWd, void* ws, size_t ws_bytes,
+                        cudaStream_t stream) {
+  int rc = check_ffn("moe_grouped_ffn_bwd", dtype, rows, E, d, f);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!xp || !Wg || !Wu || !Wd || !h1 || !h2 || !a || !dyp || !expert_offsets || !dxp || !dWg ||
+      !dWu || !dWd || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: null pointer");
+  const void* ptrs[] = {xp, Wg, Wu, Wd, h1, h2, a, dyp, dxp, dWg, dWu, dWd, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: 16-byte alignment");
+  if (ws_bytes < moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_bwd: workspace needs %zu bytes (got %zu)",
+                moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype), ws_bytes);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t h = align256(static_cast<size_t>(rows) * f * elem_bytes(dtype));
+  moe::FfnBwdArgs args{xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, rows, E, d, f, dxp,
+                       dWg, dWu, dWd, base + moe::kWsHeader, base + moe::kWsHeader + h,
+                       static_cast<unsigned*>(ws)};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_bwd_bf16(args, stream)
+                                    : moe::launch_ffn_bwd_f32(args, stream);
+  return cuda_status(e, "moe_grouped_ffn_bwd");
+}
+
+}  // extern "C"

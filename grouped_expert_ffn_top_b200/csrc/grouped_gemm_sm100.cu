@@ -1,0 +1,690 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (sm_100a):
+// tcgen05.mma with fp32 accumulators in TMEM, operands staged by TMA into
+// 128-byte-swizzled shared memory, one persistent CTA per SM walking a tile
+// list built on the device from the expert offsets (no host synchronisation;
+// an expert with no rows contributes no tile).
+// (Grouped expert compute / grouped-GEMM: leap-finetune PR #26 Summary; ART
+// issue #917 Related.)
+//
+// One kernel template serves the five GEMMs of the layer:
+//   kFwdGateUp      [h1 | h2] = xp [Wg_e | Wu_e]^T, epilogue a = silu(h1) h2
+//   kFwdDown        yp = a Wd_e^T
+//   kBwdDgradDown   da = dyp Wd_e, epilogue dh1 = da h2 silu'(h1), dh2 = da silu(h1)
+//   kBwdDgradGateUp dxp = [dh1 | dh2] [Wg_e ; Wu_e]          (K = 2f)
+//   kWgrad          dWg_e += dh1^T xp, dWu_e += dh2^T xp, dWd_e^T += a^T dyp
+// The first four have a ragged M (the expert's rows, tiles of 128; rows of a
+// tile past the expert's end are computed and discarded). kWgrad has a ragged
+// K (the expert's rows): in the last K block the rows past the expert's end
+// are zeroed in shared memory before the MMA reads them.
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM
+// and issues tcgen05.mma (one lane), warps 2-5 run the epilogue, each on its
+// TMEM lane quarter (warp % 4). Two TMEM accumulators let the epilogue of one
+// tile overlap the main loop of the next.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace moe {
+namespace gg {
+
+using namespace sm100;
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
+constexpr int kThreads = 192;
+constexpr int kMaxE = MOE_MAX_EXPERTS;
+constexpr long long kWaitLimit = 2000000000LL;  // about one second of SM cycles
+constexpr uint32_t kTmemCols = 512;
+
+enum Kind : int {
+  kFwdGateUp = 0,
+  kFwdDown = 1,
+  kBwdDgradDown = 2,
+  kBwdDgradGateUp = 3,
+  kWgrad = 4
+};
+
+struct Maps {
+  CUtensorMap a0, a1, a2, b0, b1;
+};
+
+struct Params {
+  const int64_t* offsets;
+  int E, d, f;
+  bf16* o0;
+  bf16* o1;
+  bf16* o2;
+  const bf16* i0;
+  const bf16* i1;
+  float* w0;
+  float* w1;
+  float* w2;
+  unsigned* err;
+};
+
+template <int KIND, int BN>
+struct Traits {
+  static constexpr bool A_MN = KIND == kWgrad;
+  static constexpr bool B_MN = KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || KIND == kWgrad;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;
+  static constexpr uint32_t B_BYTES = BN * BK * 2;
+  static constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
+  static constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, A_MN, B_MN);
+  // N extent of one output tile (gate/up: 128 f columns, each with its gate
+  // and up accumulator, together the MMA's N = 256)
+  static constexpr int NTILE = KIND == kFwdGateUp ? 128 : BN;
+  static constexpr size_t BAR_BYTES = 256;
+  static constexpr size_t SCHED_BYTES = 8 * (kMaxE + 1) + 4 * (kMaxE + 1) + 4 * kMaxE;
+  static constexpr size_t SMEM =
+      1024 + STAGES * static_cast<size_t>(A_BYTES + B_BYTES) + BAR_BYTES + SCHED_BYTES;
+  static_assert(KIND != kFwdGateUp || BN == 256, "gate/up pairs two 128-column accumulators");
+  static_assert(2 * BN <= static_cast<int>(kTmemCols), "two accumulators must fit in TMEM");
+  static_assert(BN % 64 == 0 && BN <= 256, "BN");
+};
+
+struct TileInfo {
+  int e;
+  int row0;  // first row of the tile (M-ragged) or of the expert (wgrad)
+  int rows;  // valid rows in the tile (M-ragged) or the expert's row count (wgrad)
+  int m0;    // wgrad: first f index of the tile
+  int n0;    // first output column of the tile
+  int prod;  // wgrad: 0 dWg, 1 dWu, 2 dWd
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+template <int KIND, int BN>
+__device__ __forceinline__ int tiles_of_expert(int cnt, int d, int f) {
+  using Tr = Traits<KIND, BN>;
+  if (cnt <= 0) return 0;
+  if (KIND == kWgrad) return 3 * ceil_div(f, BM) * ceil_div(d, BN);
+  const int n_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? f : d;
+  return ceil_div(cnt, BM) * ceil_div(n_extent, Tr::NTILE);
+}
+
+template <int KIND, int BN>
+__device__ __forceinline__ int num_kblocks(const TileInfo& ti, int d, int f) {
+  if (KIND == kFwdGateUp || KIND == kBwdDgradDown) return d / BK;
+  if (KIND == kFwdDown) return f / BK;
+  if (KIND == kBwdDgradGateUp) return 2 * (f / BK);
+  return ceil_div(ti.rows, BK);  // wgrad: ragged K
+}
+
+struct Sched {
+  const int64_t* off;  // [E+1] shared copy of the offsets
+  const int* tstart;   // [E+1] first tile of each scheduled slot
+  const int* order;    // [E] expert of each slot
+  int E;
+};
+
+template <int KIND, int BN>
+__device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d, int f) {
+  using Tr = Traits<KIND, BN>;
+  int lo = 0, hi = s.E - 1;
+  while (lo < hi) {  // largest slot whose first tile is <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.tstart[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.e = s.order[lo];
+  const int local = tile - s.tstart[lo];
+  const int base = static_cast<int>(s.off[ti.e]);
+  const int cnt = static_cast<int>(s.off[ti.e + 1] - s.off[ti.e]);
+  if (KIND == kWgrad) {
+    const int nt = ceil_div(d, BN), mt = ceil_div(f, BM);
+    ti.prod = local / (mt * nt);
+    const int rem = local % (mt * nt);
+    ti.m0 = (rem / nt) * BM;
+    ti.n0 = (rem % nt) * BN;
+    ti.row0 = base;
+    ti.rows = cnt;
+  } else {
+    const int n_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? f : d;
+    const int nt = ceil_div(n_extent, Tr::NTILE);
+    const int mi = local / nt;
+    ti.n0 = (local % nt) * Tr::NTILE;
+    ti.row0 = base + mi * BM;
+    ti.rows = min(BM, cnt - mi * BM);
+    ti.m0 = 0;
+    ti.prod = 0;
+  }
+  return ti;
+}
+
+// TMA loads of k block `kb` of tile `ti` into one pipeline stage.
+template <int KIND, int BN>
+__device__ __forceinline__ void issue_loads(const Maps& m, const TileInfo& ti, int kb, int d,
+                                            int f, uint8_t* a_dst, uint8_t* b_dst,
+                                            uint64_t* bar) {
+  const int k0 = kb * BK;
+  if (KIND == kFwdGateUp) {
+    tma_load_2d(a_dst, &m.a0, bar, k0, ti.row0);
+    const int wrow = ti.e * f + ti.n0;
+    tma_load_2d(b_dst, &m.b0, bar, k0, wrow);
+    tma_load_2d(b_dst + 128 * 128, &m.b1, bar, k0, wrow);
+  } else if (KIND == kFwdDown) {
+    tma_load_2d(a_dst, &m.a0, bar, k0, ti.row0);
+    tma_load_2d(b_dst, &m.b0, bar, k0, ti.e * d + ti.n0);
+  } else if (KIND == kBwdDgradDown) {
+    tma_load_2d(a_dst, &m.a0, bar, k0, ti.row0);
+#pragma unroll
+    for (int j = 0; j < BN / 64; ++j)
+      tma_load_2d(b_dst + j * 8192, &m.b0, bar, ti.n0 + 64 * j, ti.e * d + k0);
+  } else if (KIND == kBwdDgradGateUp) {
+    const int half = f / BK;
+    const bool second = kb >= half;
+    const int kk = (second ? kb - half : kb) * BK;
+    tma_load_2d(a_dst, second ? &m.a1 : &m.a0, bar, kk, ti.row0);
+#pragma unroll
+    for (int j = 0; j < BN / 64; ++j)
+      tma_load_2d(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + 64 * j, ti.e * f + kk);
+  } else {  // kWgrad
+    const CUtensorMap* am = ti.prod == 0 ? &m.a0 : (ti.prod == 1 ? &m.a1 : &m.a2);
+    const CUtensorMap* bm = ti.prod == 2 ? &m.b1 : &m.b0;
+    const int r = ti.row0 + k0;
+    tma_load_2d(a_dst, am, bar, ti.m0, r);
+    tma_load_2d(a_dst + 8192, am, bar, ti.m0 + 64, r);
+#pragma unroll
+    for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, bm, bar, ti.n0 + 64 * j, r);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(const float* v) {
+  uint4 o;
+  __nv_bfloat162 t0 = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 t1 = __floats2bfloat162_rn(v[2], v[3]);
+  __nv_bfloat162 t2 = __floats2bfloat162_rn(v[4], v[5]);
+  __nv_bfloat162 t3 = __floats2bfloat162_rn(v[6], v[7]);
+  o.x = *reinterpret_cast<uint32_t*>(&t0);
+  o.y = *reinterpret_cast<uint32_t*>(&t1);
+  o.z = *reinterpret_cast<uint32_t*>(&t2);
+  o.w = *reinterpret_cast<uint32_t*>(&t3);
+  return o;
+}
+
+__device__ __forceinline__ void unpack8_bf16(uint4 u, float* v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f2 = __bfloat1622float2(h[i]);
+    v[2 * i] = f2.x;
+    v[2 * i + 1] = f2.y;
+  }
+}
+
+__device__ __forceinline__ void store16_bf16(bf16* dst, const float* v) {
+  uint4* p = reinterpret_cast<uint4*>(dst);
+  p[0] = pack8_bf16(v);
+  p[1] = pack8_bf16(v + 8);
+}
+
+// Epilogue of one tile for this thread's accumulator row r.
+template <int KIND, int BN>
+__device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, uint32_t tacc,
+                                         int r) {
+  const int d = p.d, f = p.f;
+  uint32_t u[16];
+  float v[16];
+  if (KIND == kFwdGateUp) {
+    const bool valid = r < ti.rows;
+    const int64_t row = static_cast<int64_t>(ti.row0) + r;
+    for (int c = 0; c < 128; c += 16) {
+      uint32_t g[16];
+      tmem_ld16(tacc + c, g);
+      tmem_ld16(tacc + 128 + c, u);
+      tmem_ld_wait();
+      if (valid && ti.n0 + c < f) {
+        float h1[16], h2[16], a[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          h1[i] = __uint_as_float(g[i]);
+          h2[i] = __uint_as_float(u[i]);
+          a[i] = silu_f(h1[i]) * h2[i];
+        }
+        const int64_t off = row * f + ti.n0 + c;
+        store16_bf16(p.o0 + off, h1);
+        store16_bf16(p.o1 + off, h2);
+        store16_bf16(p.o2 + off, a);
+      }
+    }
+  } else if (KIND == kFwdDown || KIND == kBwdDgradGateUp) {
+    const bool valid = r < ti.rows;
+    const int64_t row = static_cast<int64_t>(ti.row0) + r;
+    for (int c = 0; c < BN; c += 16) {
+      tmem_ld16(tacc + c, u);
+      tmem_ld_wait();
+      if (valid && ti.n0 + c < d) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(u[i]);
+        store16_bf16(p.o0 + row * d + ti.n0 + c, v);
+      }
+    }
+  } else if (KIND == kBwdDgradDown) {
+    const bool valid = r < ti.rows;
+    const int64_t row = static_cast<int64_t>(ti.row0) + r;
+    for (int c = 0; c < BN; c += 16) {
+      tmem_ld16(tacc + c, u);
+      tmem_ld_wait();
+      if (valid && ti.n0 + c < f) {
+        const int64_t off = row * f + ti.n0 + c;
+        const uint4* ph1 = reinterpret_cast<const uint4*>(p.i0 + off);
+        const uint4* ph2 = reinterpret_cast<const uint4*>(p.i1 + off);
+        float h1[16], h2[16], dh1[16], dh2[16];
+        unpack8_bf16(__ldg(ph1), h1);
+        unpack8_bf16(__ldg(ph1 + 1), h1 + 8);
+        unpack8_bf16(__ldg(ph2), h2);
+        unpack8_bf16(__ldg(ph2 + 1), h2 + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float da = __uint_as_float(u[i]);
+          const float s = sigmoid_f(h1[i]);
+          dh1[i] = da * h2[i] * s * (1.0f + h1[i] * (1.0f - s));
+          dh2[i] = da * h1[i] * s;
+        }
+        store16_bf16(p.o0 + off, dh1);
+        store16_bf16(p.o1 + off, dh2);
+      }
+    }
+  } else {  // kWgrad
+    const int m = ti.m0 + r;  // f index
+    const bool valid = m < f;
+    if (ti.prod < 2) {
+      float* out = (ti.prod == 0 ? p.w0 : p.w1) + static_cast<int64_t>(ti.e) * f * d +
+                   static_cast<int64_t>(m) * d;
+      for (int c = 0; c < BN; c += 16) {
+        tmem_ld16(tacc + c, u);
+        tmem_ld_wait();
+        if (valid && ti.n0 + c < d) {
+          float4* o4 = reinterpret_cast<float4*>(out + ti.n0 + c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float4 cur = o4[q];
+            cur.x += __uint_as_float(u[4 * q + 0]);
+            cur.y += __uint_as_float(u[4 * q + 1]);
+            cur.z += __uint_as_float(u[4 * q + 2]);
+            cur.w += __uint_as_float(u[4 * q + 3]);
+            o4[q] = cur;
+          }
+        }
+      }
+    } else {
+      // dWd_e is [d, f]: this row m is column m of it; lanes hold consecutive
+      // m, so each of the 16 updates is one coalesced 128-byte access per warp
+      float* out = p.w2 + static_cast<int64_t>(ti.e) * d * f + m;
+      for (int c = 0; c < BN; c += 16) {
+        tmem_ld16(tacc + c, u);
+        tmem_ld_wait();
+        if (valid && ti.n0 + c < d) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float* q = out + static_cast<int64_t>(ti.n0 + c + i) * f;
+            *q += __uint_as_float(u[i]);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int KIND, int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
+  using Tr = Traits<KIND, BN>;
+  constexpr int STAGES = Tr::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * Tr::A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Tr::B_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* aux = tempty + 2;
+  uint64_t* drain = aux + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  int* s_total = const_cast<int*>(s_abort) + 1;
+  int64_t* s_off = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(bars) + Tr::BAR_BYTES);
+  int* s_tstart = reinterpret_cast<int*>(s_off + kMaxE + 1);
+  int* s_order = s_tstart + kMaxE + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int E = p.E, d = p.d, f = p.f;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(aux, 1);
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    // only the maps this kind fills in
+    tma_prefetch_desc(&maps.a0);
+    tma_prefetch_desc(&maps.b0);
+    if (KIND == kBwdDgradGateUp || KIND == kWgrad) tma_prefetch_desc(&maps.a1);
+    if (KIND == kFwdGateUp || KIND == kBwdDgradGateUp || KIND == kWgrad) tma_prefetch_desc(&maps.b1);
+    if (KIND == kWgrad) tma_prefetch_desc(&maps.a2);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int e = threadIdx.x; e <= E; e += kThreads) s_off[e] = p.offsets[e];
+  __syncthreads();
+  // schedule order: wgrad tiles have ragged K, so experts go longest first
+  for (int e = threadIdx.x; e < E; e += kThreads) {
+    if (KIND == kWgrad) {
+      const int64_t c = s_off[e + 1] - s_off[e];
+      int rank = 0;
+      for (int e2 = 0; e2 < E; ++e2) {
+        const int64_t c2 = s_off[e2 + 1] - s_off[e2];
+        rank += (c2 > c) || (c2 == c && e2 < e);
+      }
+      s_order[rank] = e;
+    } else {
+      s_order[e] = e;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int s0 = 0; s0 < E; s0 += 32) {
+      const int s = s0 + lane;
+      int v = 0;
+      if (s < E) {
+        const int e = s_order[s];
+        v = tiles_of_expert<KIND, BN>(static_cast<int>(s_off[e + 1] - s_off[e]), d, f);
+      }
+      int inc = v;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += o;
+      }
+      if (s < E) s_tstart[s] = carry + inc - v;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) {
+      s_tstart[E] = carry;
+      *s_total = carry;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total = *s_total;
+  const Sched sched{s_off, s_tstart, s_order, E};
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0, aux_phase = 0;
+    uint32_t issued_mask = 0, issued_par = 0;  // last load issued on full[s], and its phase
+    bool aux_pending = false;
+    for (int tile = blockIdx.x; tile < total && !*s_abort; tile += gridDim.x) {
+      const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
+      const int nk = num_kblocks<KIND, BN>(ti, d, f);
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, kWaitLimit)) break;
+        uint8_t* a_dst = sA + stage * Tr::A_BYTES;
+        uint8_t* b_dst = sB + stage * Tr::B_BYTES;
+        const bool tail = (KIND == kWgrad) && ((kb + 1) * BK > ti.rows);
+        uint64_t* bar = tail ? aux : &full[stage];
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar, Tr::STAGE_TX);
+          issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, bar);
+        }
+        if (!tail) {
+          issued_mask |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        }
+        if (tail) {
+          // rows past the expert's end belong to the next expert (or lie past
+          // the tensor): zero them in both operands so they add nothing
+          aux_pending = true;
+          if (!wait_bounded(aux, aux_phase, s_abort, kWaitLimit)) break;
+          aux_pending = false;
+          aux_phase ^= 1u;
+          const int valid = ti.rows - kb * BK;
+          const int chunks = (BK - valid) * 8;  // 16-byte chunks per 8 KB box
+          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+          for (int box = 0; box < 2 + BN / 64; ++box) {
+            uint8_t* base = (box < 2 ? a_dst + box * 8192 : b_dst + (box - 2) * 8192) + valid * 128;
+            for (int c = lane; c < chunks; c += 32) reinterpret_cast<uint4*>(base)[c] = z;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[stage]);
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (*s_abort) {
+      // leave no copy in flight into shared memory this CTA is about to free
+      volatile int never = 0;
+      for (int s = 0; s < STAGES; ++s)
+        if ((issued_mask >> s) & 1u) wait_bounded(&full[s], (issued_par >> s) & 1u, &never, kWaitLimit);
+      if (aux_pending) wait_bounded(aux, aux_phase, &never, kWaitLimit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total && !*s_abort; tile += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
+      const int nk = num_kblocks<KIND, BN>(ti, d, f);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, s_abort, kWaitLimit)) break;
+      tc_fence_after();
+      const uint32_t dtm = tmem_base + acc * BN;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bounded(&full[stage], phase, s_abort, kWaitLimit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t adesc = Tr::A_MN ? umma_desc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                            : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bdesc = Tr::B_MN ? umma_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                            : umma_desc_sw128(b_addr + kk * 32, 16, 1024);
+            mma_bf16(dtm, adesc, bdesc, Tr::IDESC, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(&tfull[acc]);
+      __syncwarp();
+    }
+    // every MMA this thread issued has completed once `drain` flips
+    if (lane == 0) mma_commit(drain);
+    __syncwarp();
+    volatile int never = 0;
+    wait_bounded(drain, 0, &never, kWaitLimit);
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total && !*s_abort; tile += gridDim.x, ++it) {
+      const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!wait_bounded(&tfull[acc], acc_phase, s_abort, kWaitLimit)) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+      epilogue<KIND, BN>(p, ti, tacc, r);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *s_abort) raise_error(p.err, kErrTimeout);
+}
+
+// ------------------------------------------------------------------ host
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor [outer, inner] (inner contiguous, row pitch `pitch` elements),
+// box [box_outer, box_inner], 128-byte swizzle, out-of-bounds reads as zero.
+static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t pitch, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int KIND, int BN>
+static cudaError_t launch(const Maps& m, const Params& p, cudaStream_t s) {
+  using Tr = Traits<KIND, BN>;
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<KIND, BN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(Tr::SMEM));
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<KIND, BN><<<sm_count(), kThreads, Tr::SMEM, s>>>(m, p);
+  return cudaGetLastError();
+}
+
+}  // namespace gg
+
+cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
+  using namespace gg;
+  const uint64_t rows = static_cast<uint64_t>(a.rows), E = a.E, d = a.d, f = a.f;
+  Params p{};
+  p.offsets = a.offsets;
+  p.E = a.E;
+  p.d = a.d;
+  p.f = a.f;
+  p.err = a.err;
+  Maps m1{};
+  if (!make_map(&m1.a0, a.xp, d, rows, d, 64, 128) || !make_map(&m1.b0, a.Wg, d, E * f, d, 64, 128) ||
+      !make_map(&m1.b1, a.Wu, d, E * f, d, 64, 128))
+    return cudaErrorInvalidValue;
+  p.o0 = static_cast<bf16*>(a.h1);
+  p.o1 = static_cast<bf16*>(a.h2);
+  p.o2 = static_cast<bf16*>(a.a);
+  cudaError_t e = launch<kFwdGateUp, 256>(m1, p, s);
+  if (e != cudaSuccess) return e;
+  Maps m2{};
+  if (!make_map(&m2.a0, a.a, f, rows, f, 64, 128) || !make_map(&m2.b0, a.Wd, f, E * d, f, 64, 256))
+    return cudaErrorInvalidValue;
+  p.o0 = static_cast<bf16*>(a.yp);
+  p.o1 = p.o2 = nullptr;
+  return launch<kFwdDown, 256>(m2, p, s);
+}
+
+cudaError_t launch_ffn_bwd_bf16(const FfnBwdArgs& a, cudaStream_t s) {
+  using namespace gg;
+  const uint64_t rows = static_cast<uint64_t>(a.rows), E = a.E, d = a.d, f = a.f;
+  Params p{};
+  p.offsets = a.offsets;
+  p.E = a.E;
+  p.d = a.d;
+  p.f = a.f;
+  p.err = a.err;
+  // 1. da = dyp Wd_e, SwiGLU backward in the epilogue -> dh1, dh2
+  Maps m1{};
+  if (!make_map(&m1.a0, a.dyp, d, rows, d, 64, 128) || !make_map(&m1.b0, a.Wd, f, E * d, f, 64, 64))
+    return cudaErrorInvalidValue;
+  p.i0 = static_cast<const bf16*>(a.h1);
+  p.i1 = static_cast<const bf16*>(a.h2);
+  p.o0 = static_cast<bf16*>(a.dh1);
+  p.o1 = static_cast<bf16*>(a.dh2);
+  cudaError_t e = (a.f % 256 == 0) ? launch<kBwdDgradDown, 256>(m1, p, s)
+                                   : launch<kBwdDgradDown, 128>(m1, p, s);
+  if (e != cudaSuccess) return e;
+  // 2. dxp = dh1 Wg_e + dh2 Wu_e
+  Maps m2{};
+  if (!make_map(&m2.a0, a.dh1, f, rows, f, 64, 128) || !make_map(&m2.a1, a.dh2, f, rows, f, 64, 128) ||
+      !make_map(&m2.b0, a.Wg, d, E * f, d, 64, 64) || !make_map(&m2.b1, a.Wu, d, E * f, d, 64, 64))
+    return cudaErrorInvalidValue;
+  p.i0 = p.i1 = nullptr;
+  p.o0 = static_cast<bf16*>(a.dxp);
+  p.o1 = nullptr;
+  e = launch<kBwdDgradGateUp, 256>(m2, p, s);
+  if (e != cudaSuccess) return e;
+  // 3. weight gradients, accumulated in fp32
+  Maps m3{};
+  if (!make_map(&m3.a0, a.dh1, f, rows, f, 64, 64) || !make_map(&m3.a1, a.dh2, f, rows, f, 64, 64) ||
+      !make_map(&m3.a2, a.a, f, rows, f, 64, 64) || !make_map(&m3.b0, a.xp, d, rows, d, 64, 64) ||
+      !make_map(&m3.b1, a.dyp, d, rows, d, 64, 64))
+    return cudaErrorInvalidValue;
+  p.o0 = nullptr;
+  p.w0 = a.dWg;
+  p.w1 = a.dWu;
+  p.w2 = a.dWd;
+  return launch<kWgrad, 256>(m3, p, s);
+}
+
+}  // namespace moe

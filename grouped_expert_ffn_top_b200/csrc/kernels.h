@@ -1,0 +1,66 @@
+// Internal launchers of the MoE layer library (host side, no validation:
+// the C ABI in api.cu checks every argument before calling these).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kRouteThreads = 256;
+constexpr int kRouteTokensPerBlock = 256;
+
+// routing (route.cu)
+cudaError_t launch_router_logits(const void* x, const void* Wr, const float* b, int dtype,
+                                 int64_t T, int d, int E, float* z, cudaStream_t s);
+cudaError_t launch_route(const float* z, int64_t T, int E, int k, int G, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, int64_t* offsets, int32_t* group_counts,
+                         int64_t* group_offsets, int32_t* row_of_pair, int32_t* pair_of_row,
+                         int32_t* block_counts, int32_t* block_base, unsigned* err,
+                         cudaStream_t s);
+cudaError_t route_set_smem_limits();
+cudaError_t launch_route_bwd(const float* dg, const float* w, const int32_t* idx, int64_t T,
+                             int E, int k, float* dz, cudaStream_t s);
+
+// dispatch / combine (dispatch.cu)
+cudaError_t launch_permute(const void* x, int dtype, int64_t T, int d, int k,
+                           const int32_t* row_of_pair, void* xp, cudaStream_t s);
+cudaError_t launch_combine(const void* yp, const float* w, const int32_t* row_of_pair, int dtype,
+                           int64_t T, int d, int k, void* Y, cudaStream_t s);
+cudaError_t launch_combine_bwd(const void* dY, const void* yp, const float* w,
+                               const int32_t* row_of_pair, int dtype, int64_t T, int d, int k,
+                               void* dyp, float* dg, cudaStream_t s);
+cudaError_t launch_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dz,
+                               const void* Wr, const int32_t* idx, int dtype, int64_t T, int d,
+                               int E, int k, void* dX, cudaStream_t s);
+int router_bwd_splits(int64_t T, int d, int E);
+cudaError_t launch_router_bwd(const void* x, const float* dz, int dtype, int64_t T, int d, int E,
+                              float* dWr, float* db, float* partial, cudaStream_t s);
+
+// grouped expert FFN (grouped_gemm_sm100.cu, grouped_simt.cu)
+struct FfnFwdArgs {
+  const void *xp, *Wg, *Wu, *Wd;
+  const int64_t* offsets;
+  int64_t rows;
+  int E, d, f;
+  void *h1, *h2, *a, *yp;
+  unsigned* err;
+};
+struct FfnBwdArgs {
+  const void *xp, *Wg, *Wu, *Wd, *h1, *h2, *a, *dyp;
+  const int64_t* offsets;
+  int64_t rows;
+  int E, d, f;
+  void* dxp;
+  float *dWg, *dWu, *dWd;
+  void *dh1, *dh2;  // scratch [rows, f]
+  unsigned* err;
+};
+
+cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_bwd_bf16(const FfnBwdArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_fwd_f32(const FfnFwdArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_bwd_f32(const FfnBwdArgs& a, cudaStream_t s);
+
+}  // namespace moe

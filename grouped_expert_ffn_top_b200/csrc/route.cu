@@ -1,0 +1,412 @@
+// Routing kernels: router logits, top-k softmax, the per-expert histogram /
+// scan / stable scatter that builds the dispatch layout, and the route
+// backward. (Expert routing and EP token dispatch: ART issue #917 intro and
+// Desired behavior; leap-finetune PR #26 Summary.)
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// ------------------------------------------------------------ router logits
+//
+// z[t,e] = fma-chain over i = 0..d-1 of x[t,i] * Wr[e,i], then + b[e], in fp32.
+// Block tile: 128 tokens x TE experts; thread tile: 8 tokens x TE/8 experts.
+// Both operands are staged in shared memory as fp32, i-major, so one thread
+// reads 8 consecutive tokens and TE/8 consecutive experts with 128-bit loads.
+// The i loop is sequential for every output, which is what makes the result
+// bit-identical to the fixed-order definition.
+
+constexpr int kLogitTokens = 128;
+constexpr int kLogitChunk = 32;
+
+template <typename T, int TE>
+__global__ void __launch_bounds__(128) router_logits_kernel(const T* __restrict__ x,
+                                                            const T* __restrict__ Wr,
+                                                            const float* __restrict__ b,
+                                                            int64_t Ttok, int d, int E,
+                                                            float* __restrict__ z) {
+  constexpr int EPT = TE / 8;  // experts per thread
+  __shared__ __align__(16) float xs[kLogitChunk][kLogitTokens];
+  __shared__ __align__(16) float ws[kLogitChunk][TE];
+  const int tid = threadIdx.x;
+  const int tx = tid % 8;   // expert group
+  const int ty = tid / 8;   // token group (16 of them)
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kLogitTokens;
+  const int e0 = blockIdx.y * TE;
+
+  float acc[8][EPT];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < EPT; ++c) acc[a][c] = 0.0f;
+
+  for (int i0 = 0; i0 < d; i0 += kLogitChunk) {
+    // stage x[t0 .. t0+127][i0 .. i0+31] transposed into xs[i][t]
+    // consecutive threads take consecutive tokens: conflict-free shared stores;
+    // the strided global reads of one row are served from L1 across ii
+    for (int idx = tid; idx < kLogitTokens * kLogitChunk; idx += 128) {
+      int tt = idx % kLogitTokens, ii = idx / kLogitTokens;
+      int64_t t = t0 + tt;
+      int i = i0 + ii;
+      xs[ii][tt] = (t < Ttok && i < d) ? to_f32(x[t * d + i]) : 0.0f;
+    }
+    for (int idx = tid; idx < TE * kLogitChunk; idx += 128) {
+      int ee = idx % TE, ii = idx / TE;
+      int e = e0 + ee, i = i0 + ii;
+      ws[ii][ee] = (e < E && i < d) ? to_f32(Wr[static_cast<int64_t>(e) * d + i]) : 0.0f;
+    }
+    __syncthreads();
+    const int iend = min(kLogitChunk, d - i0);
+    for (int ii = 0; ii < iend; ++ii) {
+      float xv[8], wv[EPT];
+      const float4 xa = *reinterpret_cast<const float4*>(&xs[ii][ty * 8]);
+      const float4 xb = *reinterpret_cast<const float4*>(&xs[ii][ty * 8 + 4]);
+      xv[0] = xa.x; xv[1] = xa.y; xv[2] = xa.z; xv[3] = xa.w;
+      xv[4] = xb.x; xv[5] = xb.y; xv[6] = xb.z; xv[7] = xb.w;
+#pragma unroll
+      for (int c = 0; c < EPT; ++c) wv[c] = ws[ii][tx * EPT + c];
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int c = 0; c < EPT; ++c) acc[a][c] = __fmaf_rn(xv[a], wv[c], acc[a][c]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int a = 0; a < 8; ++a) {
+    const int64_t t = t0 + ty * 8 + a;
+    if (t >= Ttok) continue;
+#pragma unroll
+    for (int c = 0; c < EPT; ++c) {
+      const int e = e0 + tx * EPT + c;
+      if (e < E) z[t * E + e] = __fadd_rn(acc[a][c], b ? b[e] : 0.0f);
+    }
+  }
+}
+
+template <typename T>
+static cudaError_t launch_router_logits_t(const T* x, const T* Wr, const float* b, int64_t Ttok,
+                                          int d, int E, float* z, cudaStream_t s) {
+  const unsigned gx = static_cast<unsigned>((Ttok + kLogitTokens - 1) / kLogitTokens);
+  if (E <= 8) {
+    router_logits_kernel<T, 8><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+  } else if (E <= 16) {
+    router_logits_kernel<T, 16><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+  } else if (E <= 32) {
+    router_logits_kernel<T, 32><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+  } else {
+    router_logits_kernel<T, 64><<<dim3(gx, (E + 63) / 64), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_logits(const void* x, const void* Wr, const float* b, int dtype,
+                                 int64_t T, int d, int E, float* z, cudaStream_t s) {
+  if (dtype == MOE_BF16)
+    return launch_router_logits_t(static_cast<const bf16*>(x), static_cast<const bf16*>(Wr), b, T,
+                                  d, E, z, s);
+  return launch_router_logits_t(static_cast<const float*>(x), static_cast<const float*>(Wr), b, T,
+                                d, E, z, s);
+}
+
+// ------------------------------------------------------------------- top-k
+//
+// One warp per token. Lane l holds the logits of experts l, l+32, ...; k
+// rounds of a warp arg-max pick the experts in ranking order (larger logit
+// first, NaN after every number, lower index on equal keys). The block's 256
+// tokens are also counted per expert (shared-memory histogram) for the scan.
+
+struct Cand {
+  float v;
+  int idx;  // INT_MAX when the slot is empty or already taken
+};
+
+__device__ __forceinline__ bool ranks_before(const Cand& a, const Cand& b) {
+  const bool ea = a.idx == INT_MAX, eb = b.idx == INT_MAX;
+  if (ea != eb) return eb;
+  const bool na = isnan(a.v), nb = isnan(b.v);
+  if (na != nb) return nb;
+  if (!na && a.v != b.v) return a.v > b.v;
+  return a.idx < b.idx;
+}
+
+template <int S>  // S = ceil(E / 32) logits per lane
+__global__ void __launch_bounds__(kRouteThreads) topk_softmax_kernel(
+    const float* __restrict__ z, int64_t Ttok, int E, int k, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w, int32_t* __restrict__ block_counts, unsigned* err) {
+  extern __shared__ int s_hist[];  // [E]
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+
+  const int64_t tok_base = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock;
+  constexpr int kTokPerWarp = kRouteTokensPerBlock / (kRouteThreads / 32);
+  for (int q = 0; q < kTokPerWarp; ++q) {
+    const int64_t t = tok_base + warp * kTokPerWarp + q;
+    if (t >= Ttok) break;
+    float v[S];
+    bool taken[S];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      const int e = lane + 32 * s;
+      v[s] = e < E ? z[t * E + e] : 0.0f;
+      taken[s] = e >= E;
+    }
+    float my_val = 0.0f;  // lane j keeps the j-th selected logit
+    int my_idx = 0;
+    for (int j = 0; j < k; ++j) {
+      Cand best{0.0f, INT_MAX};
+#pragma unroll
+      for (int s = 0; s < S; ++s) {
+        Cand c{v[s], taken[s] ? INT_MAX : lane + 32 * s};
+        if (ranks_before(c, best)) best = c;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        Cand o;
+        o.v = __shfl_xor_sync(0xffffffffu, best.v, off);
+        o.idx = __shfl_xor_sync(0xffffffffu, best.idx, off);
+        if (ranks_before(o, best)) best = o;
+      }
+      // every lane now holds the same winner; its owner marks it taken
+      if ((best.idx & 31) == lane) {
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+          if (lane + 32 * s == best.idx) taken[s] = true;
+      }
+      if (lane == j) {
+        my_val = best.v;
+        my_idx = best.idx;
+      }
+    }
+    // softmax over the k selected logits (fp32)
+    const bool active = lane < k;
+    const bool finite = !active || isfinite(my_val);
+    const bool all_finite = __all_sync(0xffffffffu, finite);
+    const float m = __shfl_sync(0xffffffffu, my_val, 0);
+    float ex = (active && all_finite) ? expf(my_val - m) : 0.0f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (active) {
+      const float w = all_finite ? ex / sum : 1.0f / static_cast<float>(k);
+      topk_idx[t * k + lane] = my_idx;
+      topk_w[t * k + lane] = w;
+      atomicAdd(&s_hist[my_idx], 1);
+    }
+    if (!all_finite && lane == 0) raise_error(err, kErrNonfiniteLogit);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    block_counts[static_cast<int64_t>(blockIdx.x) * E + e] = s_hist[e];
+}
+
+// --------------------------------------------------------------------- scan
+//
+// One block. totals[e] = sum over blocks; offsets = exclusive scan of totals;
+// block_base[b][e] = offsets[e] + sum_{b' < b} block_counts[b'][e]; group
+// counts and offsets from contiguous expert blocks.
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    int o = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += o;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(1024) route_scan_kernel(
+    const int32_t* __restrict__ block_counts, int nb, int E, int G,
+    int32_t* __restrict__ block_base, int32_t* __restrict__ counts, int64_t* __restrict__ offsets,
+    int32_t* __restrict__ group_counts, int64_t* __restrict__ group_offsets) {
+  __shared__ int s_tot[MOE_MAX_EXPERTS];
+  __shared__ int s_off[MOE_MAX_EXPERTS + 1];
+  __shared__ int s_warp[32];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  // per-expert totals
+  for (int e = warp; e < E; e += nwarps) {
+    int s = 0;
+    for (int b = lane; b < nb; b += 32) s += block_counts[static_cast<int64_t>(b) * E + e];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) s_tot[e] = s;
+  }
+  __syncthreads();
+  // exclusive scan of the totals over experts (E <= 1024 = blockDim)
+  {
+    const int e = threadIdx.x;
+    const int v = e < E ? s_tot[e] : 0;
+    const int inc = warp_incl_scan(v);
+    if (lane == 31) s_warp[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+      int wv = lane < nwarps ? s_warp[lane] : 0;
+      int winc = warp_incl_scan(wv);
+      s_warp[lane] = winc - wv;
+    }
+    __syncthreads();
+    const int excl = inc - v + s_warp[warp];
+    if (e < E) {
+      s_off[e] = excl;
+      counts[e] = v;
+      offsets[e] = excl;
+    }
+    if (e == E - 1) {
+      s_off[E] = excl + v;
+      offsets[E] = excl + v;
+    }
+  }
+  __syncthreads();
+  // absolute per-block bases
+  for (int e = warp; e < E; e += nwarps) {
+    int carry = s_off[e];
+    for (int b0 = 0; b0 < nb; b0 += 32) {
+      const int b = b0 + lane;
+      const int v = b < nb ? block_counts[static_cast<int64_t>(b) * E + e] : 0;
+      const int inc = warp_incl_scan(v);
+      if (b < nb) block_base[static_cast<int64_t>(b) * E + e] = carry + inc - v;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+  }
+  // groups: contiguous blocks of E/G experts
+  const int per = E / G;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    group_counts[g] = s_off[(g + 1) * per] - s_off[g * per];
+    group_offsets[g] = s_off[g * per];
+  }
+  if (threadIdx.x == 0) group_offsets[G] = s_off[E];
+}
+
+// ------------------------------------------------------------------ scatter
+//
+// One thread per token. In each warp, bit l of mask[warp][e] says lane l's
+// token selected e; the pair's rank among earlier tokens of the same expert
+// is (earlier warps of the block) + popc(mask & lanes below). Tokens are
+// visited in order inside a warp and warps in order inside a block, so rows
+// come out sorted by token within each expert: a stable, deterministic order
+// with no atomics deciding it.
+
+__global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t Ttok, int E, int k,
+    const int32_t* __restrict__ block_base, int32_t* __restrict__ row_of_pair,
+    int32_t* __restrict__ pair_of_row) {
+  extern __shared__ unsigned s_mem[];
+  constexpr int W = kRouteThreads / 32;
+  unsigned* mask = s_mem;                                   // [W][E]
+  int* wbase = reinterpret_cast<int*>(s_mem + W * E);       // [W][E]
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < W * E; i += blockDim.x) mask[i] = 0u;
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock + threadIdx.x;
+  const bool valid = t < Ttok;
+  if (valid)
+    for (int j = 0; j < k; ++j) atomicOr(&mask[warp * E + topk_idx[t * k + j]], 1u << lane);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < W; ++w) {
+      wbase[w * E + e] = run;
+      run += __popc(mask[w * E + e]);
+    }
+  }
+  __syncthreads();
+  if (!valid) return;
+  const unsigned below = (1u << lane) - 1u;
+  for (int j = 0; j < k; ++j) {
+    const int e = topk_idx[t * k + j];
+    const int row = block_base[static_cast<int64_t>(blockIdx.x) * E + e] + wbase[warp * E + e] +
+                    __popc(mask[warp * E + e] & below);
+    row_of_pair[t * k + j] = row;
+    pair_of_row[row] = static_cast<int32_t>(t * k + j);
+  }
+}
+
+cudaError_t launch_route(const float* z, int64_t T, int E, int k, int G, int32_t* topk_idx,
+                         float* topk_w, int32_t* counts, int64_t* offsets, int32_t* group_counts,
+                         int64_t* group_offsets, int32_t* row_of_pair, int32_t* pair_of_row,
+                         int32_t* block_counts, int32_t* block_base, unsigned* err,
+                         cudaStream_t s) {
+  const int nb = static_cast<int>((T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock);
+  const size_t hist_smem = sizeof(int) * E;
+  const int S = (E + 31) / 32;
+#define MOE_TOPK_CASE(SV)                                                                  \
+  topk_softmax_kernel<SV><<<nb, kRouteThreads, hist_smem, s>>>(z, T, E, k, topk_idx, topk_w, \
+                                                               block_counts, err)
+  if (S <= 1) MOE_TOPK_CASE(1);
+  else if (S <= 2) MOE_TOPK_CASE(2);
+  else if (S <= 4) MOE_TOPK_CASE(4);
+  else if (S <= 8) MOE_TOPK_CASE(8);
+  else if (S <= 16) MOE_TOPK_CASE(16);
+  else MOE_TOPK_CASE(32);
+#undef MOE_TOPK_CASE
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, G, block_base, counts, offsets,
+                                        group_counts, group_offsets);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t scatter_smem = sizeof(unsigned) * 2 * (kRouteThreads / 32) * E;
+  route_scatter_kernel<<<nb, kRouteThreads, scatter_smem, s>>>(topk_idx, T, E, k, block_base,
+                                                               row_of_pair, pair_of_row);
+  return cudaGetLastError();
+}
+
+cudaError_t route_set_smem_limits() {
+  const int scatter_max = static_cast<int>(sizeof(unsigned) * 2 * (kRouteThreads / 32) *
+                                           MOE_MAX_EXPERTS);
+  return cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              scatter_max);
+}
+
+// ------------------------------------------------------------ route backward
+//
+// dz[t, S_j] = g_j (dg_j - sum_m g_m dg_m); dz = 0 off the selection.
+// One warp per token; every dlogits entry is written exactly once.
+
+__global__ void __launch_bounds__(256) route_bwd_kernel(const float* __restrict__ dg,
+                                                        const float* __restrict__ w,
+                                                        const int32_t* __restrict__ idx,
+                                                        int64_t Ttok, int E, int k,
+                                                        float* __restrict__ dz) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (t >= Ttok) return;
+  float gj = 0.0f, dgj = 0.0f;
+  int ij = -1;
+  if (lane < k) {
+    gj = w[t * k + lane];
+    dgj = dg[t * k + lane];
+    ij = idx[t * k + lane];
+  }
+  float s = gj * dgj;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  const float mine = gj * (dgj - s);
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    float v = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int ie = __shfl_sync(0xffffffffu, ij, j);
+      const float dv = __shfl_sync(0xffffffffu, mine, j);
+      if (ie == e) v = dv;
+    }
+    if (e < E) dz[t * E + e] = v;
+  }
+}
+
+cudaError_t launch_route_bwd(const float* dg, const float* w, const int32_t* idx, int64_t T,
+                             int E, int k, float* dz, cudaStream_t s) {
+  const unsigned grid = static_cast<unsigned>((T + 7) / 8);
+  route_bwd_kernel<<<grid, 256, 0, s>>>(dg, w, idx, T, E, k, dz);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

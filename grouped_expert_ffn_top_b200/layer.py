@@ -1,0 +1,125 @@
+"""One MoE layer driven through the C ABI: the call sequence of a training step.
+
+Forward:  moe_router_logits -> moe_route -> moe_permute -> moe_grouped_ffn_fwd
+          -> moe_unpermute_combine
+Backward: moe_unpermute_combine_bwd -> moe_route_bwd -> moe_grouped_ffn_bwd
+          -> moe_permute_bwd (with the router's input gradient) -> moe_router_bwd
+
+The object owns device buffers sized for `max_tokens`, so a step allocates
+nothing; microbatches of any size up to that (0 included) reuse them. Weight
+gradients accumulate in fp32 across microbatches until zero_grad().
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import native as N
+
+
+class MoELayer:
+    def __init__(self, params: Dict[str, torch.Tensor], k: int, ep_groups: int = 1,
+                 max_tokens: int = 0):
+        self.Wr, self.b = params["Wr"], params["b"]
+        self.Wg, self.Wu, self.Wd = params["Wg"], params["Wu"], params["Wd"]
+        self.E, self.f, self.d = self.Wg.shape
+        self.k, self.G = k, ep_groups
+        self.dtype = self.Wg.dtype
+        self.dt = N.MOE_BF16 if self.dtype == torch.bfloat16 else N.MOE_F32
+        dev = self.Wg.device
+        self.device = dev
+        f32 = torch.float32
+        self.grads = {
+            "dWr": torch.zeros((self.E, self.d), dtype=f32, device=dev),
+            "db": torch.zeros(self.E, dtype=f32, device=dev),
+            "dWg": torch.zeros((self.E, self.f, self.d), dtype=f32, device=dev),
+            "dWu": torch.zeros((self.E, self.f, self.d), dtype=f32, device=dev),
+            "dWd": torch.zeros((self.E, self.d, self.f), dtype=f32, device=dev),
+        }
+        self.max_tokens = 0
+        self.T = 0
+        self.reserve(max(1, max_tokens))
+
+    def reserve(self, T: int) -> None:
+        """Make the buffers hold microbatches of up to T tokens."""
+        if T <= self.max_tokens:
+            return
+        dev, dt, E, k, d, f = self.device, self.dtype, self.E, self.k, self.d, self.f
+        P = T * k
+        f32 = torch.float32
+        self.buf = {
+            "logits": torch.empty((T, E), dtype=f32, device=dev),
+            "xp": torch.empty((P, d), dtype=dt, device=dev),
+            "h1": torch.empty((P, f), dtype=dt, device=dev),
+            "h2": torch.empty((P, f), dtype=dt, device=dev),
+            "a": torch.empty((P, f), dtype=dt, device=dev),
+            "yp": torch.empty((P, d), dtype=dt, device=dev),
+            "Y": torch.empty((T, d), dtype=dt, device=dev),
+            "dyp": torch.empty((P, d), dtype=dt, device=dev),
+            "dg": torch.empty((T, k), dtype=f32, device=dev),
+            "dlogits": torch.empty((T, E), dtype=f32, device=dev),
+            "dxp": torch.empty((P, d), dtype=dt, device=dev),
+            "dX": torch.empty((T, d), dtype=dt, device=dev),
+        }
+        self.route = N.route_outputs(T, E, k, self.G, dev)
+        self.ws = {
+            "route": N._ws(N.moe_route_workspace_bytes(T, E), dev),
+            "ffn_fwd": N._ws(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt), dev),
+            "ffn_bwd": N._ws(N.moe_grouped_ffn_bwd_workspace_bytes(P, E, d, f, self.dt), dev),
+            "router_bwd": N._ws(N.moe_router_bwd_workspace_bytes(T, d, E), dev),
+        }
+        self.max_tokens = T
+
+    def zero_grad(self) -> None:
+        for g in self.grads.values():
+            g.zero_()
+
+    def _views(self, T: int):
+        P = T * self.k
+        b = self.buf
+        r = self.route
+        v = {n: b[n][:T] for n in ("logits", "Y", "dg", "dlogits", "dX")}
+        v.update({n: b[n][:P] for n in ("xp", "h1", "h2", "a", "yp", "dyp", "dxp")})
+        ro = dict(r)
+        for n in ("topk_idx", "topk_w"):
+            ro[n] = r[n][:T]
+        for n in ("row_of_pair", "pair_of_row"):
+            ro[n] = r[n][:P]
+        return v, ro
+
+    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        T = x.shape[0]
+        self.reserve(T)
+        self.T = T
+        self.x = x
+        v, r = self._views(T)
+        self.v, self.r = v, r
+        N.moe_router_logits(x, self.Wr, self.b, v["logits"], stream)
+        N.moe_route(v["logits"], self.k, self.G, r, self.ws["route"], stream)
+        N.moe_permute(x, r["row_of_pair"], self.k, v["xp"], stream)
+        N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"],
+                              {n: v[n] for n in ("h1", "h2", "a", "yp")}, self.ws["ffn_fwd"], stream)
+        N.moe_unpermute_combine(v["yp"], r["topk_w"], r["row_of_pair"], v["Y"], stream)
+        return v["Y"]
+
+    def backward(self, dY: torch.Tensor, stream=None) -> torch.Tensor:
+        T = self.T
+        v, r = self.v, self.r
+        g = self.grads
+        N.moe_unpermute_combine_bwd(dY, v["yp"], r["topk_w"], r["row_of_pair"], v["dyp"], v["dg"], stream)
+        N.moe_route_bwd(v["dg"], r["topk_w"], r["topk_idx"], self.E, v["dlogits"], stream)
+        N.moe_grouped_ffn_bwd(v["xp"], self.Wg, self.Wu, self.Wd, v["h1"], v["h2"], v["a"], v["dyp"],
+                              r["offsets"], g["dWg"], g["dWu"], g["dWd"], v["dxp"], self.ws["ffn_bwd"],
+                              stream)
+        N.moe_permute_bwd(v["dxp"], r["row_of_pair"], v["dlogits"], self.Wr, r["topk_idx"], T, self.k,
+                          v["dX"], stream)
+        N.moe_router_bwd(self.x, v["dlogits"], g["dWr"], g["db"], self.ws["router_bwd"], stream)
+        return v["dX"]
+
+    def device_errors(self) -> int:
+        """Synchronises and returns (and clears) the device error words."""
+        err = 0
+        for n in ("route", "ffn_fwd", "ffn_bwd"):
+            err |= N.moe_get_error(self.ws[n])
+        return err

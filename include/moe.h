@@ -1,0 +1,248 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE layer hot path.
+ *
+ * The layer is the one the expert-parallel MoE training runtimes on the
+ * pages run on every step: expert routing, EP token dispatch, grouped expert
+ * compute, and the combine that restores full source-order outputs, forward
+ * and backward, with uneven and empty work per expert and per microbatch.
+ *   - "EP token dispatch, grouped expert compute": leap-finetune PR #26
+ *     "Add MoE expert parallel training runtime", Summary / Major changes.
+ *   - "grouped-GEMM": ART issue #917 "Support combined expert and data
+ *     parallelism in TrainerRank", Related.
+ *   - expert-routing communication, expert communication groups, full
+ *     source-order outputs, accumulation, uneven or empty work, explicit
+ *     errors for unsupported cases: ART issue #917, intro, Desired behavior
+ *     and Acceptance.
+ * The pages give no formulas; the arithmetic below is the plainest reading
+ * (a dropless top-k softmax-gated mixture of SwiGLU experts):
+ *   z      = x Wr^T + b                             router logits
+ *   S_t    = the k largest z[t,:], ties to the lower expert index, in
+ *            descending order (slot j holds the j-th largest)
+ *   g_t    = softmax(z[t, S_t])                     gate weights, sum to 1
+ *   h1 = xp Wg_e^T, h2 = xp Wu_e^T, a = silu(h1) * h2, yp = a Wd_e^T
+ *   Y_t    = sum_j g_{t,j} yp[row(t,j)]
+ * and the backward is the exact gradient of that with S_t held fixed.
+ *
+ * Conventions (every entry point):
+ *   - Pointers are DEVICE pointers unless stated otherwise, owned by the
+ *     caller. The library never allocates device memory. Scratch memory is
+ *     a caller buffer `ws` of at least the size the matching
+ *     *_workspace_bytes function returns; it must be zero-filled once after
+ *     allocation (its first bytes hold the device error word).
+ *   - Tensors are dense row-major; the last listed dimension is contiguous.
+ *   - `dtype` selects the element type of activations and weights:
+ *     MOE_BF16 (bf16 storage, fp32 accumulation, tcgen05 tensor cores) or
+ *     MOE_F32 (fp32 throughout, CUDA cores). Logits, gate weights and every
+ *     gradient of a parameter are fp32.
+ *   - Index arrays are int32; offsets are int64.
+ *   - Every call is asynchronous on `stream`, performs no host
+ *     synchronisation and no allocation. moe_get_error is the one call that
+ *     synchronises.
+ *   - T = 0 (an empty microbatch) is valid everywhere: the call returns
+ *     MOE_OK, launches nothing and leaves every output and accumulator as it
+ *     was.
+ *   - Gradients of parameters accumulate (+=) into fp32 buffers the caller
+ *     zeroes before the first microbatch; activation gradients overwrite.
+ *   - Return value: MOE_OK, or a negative MOE_ERR_* code with a message
+ *     available from moe_last_error() (thread-local). Arguments are checked
+ *     before anything is launched; a rejected call changes nothing.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_F32 0
+#define MOE_BF16 1
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1) /* null pointer, negative size, k < 1, k > E */
+#define MOE_ERR_UNSUPPORTED (-2) /* shape or dtype outside the supported set  */
+#define MOE_ERR_WORKSPACE (-3)   /* ws too small or misaligned                */
+#define MOE_ERR_CUDA (-4)        /* a CUDA call or launch failed              */
+
+/* Bits of the device error word returned by moe_get_error. */
+#define MOE_DEVERR_NONFINITE_LOGIT 1u /* a selected router logit was NaN or +-inf */
+#define MOE_DEVERR_TIMEOUT 2u         /* a bounded wait inside a kernel gave up   */
+
+/* Limits of this build. */
+#define MOE_MAX_EXPERTS 1024
+
+/* Message of the last failed call on this host thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Library ABI version (increments on any signature change). */
+MOE_API int moe_version(void);
+
+/* Synchronises `stream`, returns the device error word accumulated in `ws`
+ * by the calls that used it since the last moe_get_error (0 = no error), and
+ * clears it. Returns MOE_ERR_CUDA (< 0) if the synchronisation fails. */
+MOE_API int moe_get_error(void* ws, cudaStream_t stream);
+
+/* ------------------------------------------------------------ routing */
+
+/* Router logits z[t,e] = sum_i x[t,i] Wr[e,i] + b[e], in fp32: one fused
+ * multiply-add per element in ascending i, then one add of b[e]. This fixed
+ * order makes the logits, and therefore the top-k, bit-reproducible.
+ * (Expert-routing step: ART issue #917, intro.)
+ *   x       [T, d]   dtype      activations
+ *   Wr      [E, d]   dtype      router weight
+ *   b       [E]      fp32       router bias (may be NULL: no bias)
+ *   logits  [T, E]   fp32       output
+ * Errors: INVALID_ARG for null x/Wr/logits with T > 0 or d, E < 1;
+ * UNSUPPORTED for E > MOE_MAX_EXPERTS or d not a multiple of 8. */
+MOE_API int moe_router_logits(const void* x, const void* Wr, const float* b, int dtype,
+                      int64_t T, int d, int E, float* logits, cudaStream_t stream);
+
+/* Workspace of moe_route, in bytes. */
+MOE_API size_t moe_route_workspace_bytes(int64_t T, int E);
+
+/* Top-k softmax routing and the dispatch layout, all on the device.
+ * Selection: per token the k largest logits, ties to the lower expert index,
+ * NaN below every number, slots in descending order. Gate weights: softmax
+ * over the k selected logits (they sum to 1). If a selected logit is not
+ * finite the token's weights are 1/k each and MOE_DEVERR_NONFINITE_LOGIT is
+ * raised in the ws error word.
+ * Layout (EP token dispatch, leap-finetune PR #26 Summary; expert
+ * communication groups, ART issue #917 Desired behavior): pair (t,j) gets
+ * row row_of_pair[t*k+j]; rows are sorted by (expert, token), both
+ * ascending, so expert e owns rows [expert_offsets[e], expert_offsets[e+1])
+ * in token order (stable, dropless, no padding). Experts are split into
+ * `ep_groups` contiguous blocks of E/ep_groups (the destination groups an
+ * all-to-all would send to); group g owns rows
+ * [group_offsets[g], group_offsets[g+1]).
+ *   logits         [T, E]        fp32  input
+ *   topk_idx       [T, k]        int32 output, selected experts
+ *   topk_w         [T, k]        fp32  output, gate weights
+ *   expert_counts  [E]           int32 output
+ *   expert_offsets [E+1]         int64 output, exclusive prefix sum
+ *   group_counts   [ep_groups]   int32 output
+ *   group_offsets  [ep_groups+1] int64 output
+ *   row_of_pair    [T*k]         int32 output
+ *   pair_of_row    [T*k]         int32 output, inverse permutation
+ * For T = 0 nothing is written (as for every call), so a caller that reads
+ * the counts of an empty microbatch zeroes them itself.
+ * Errors: INVALID_ARG (null pointer, k < 1, k > E, ep_groups < 1),
+ * UNSUPPORTED (E > MOE_MAX_EXPERTS, k > 32, E % ep_groups != 0,
+ * T*k >= 2^31), WORKSPACE (ws_bytes < moe_route_workspace_bytes or ws not
+ * 16-byte aligned). */
+MOE_API int moe_route(const float* logits, int64_t T, int E, int k, int ep_groups,
+              int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
+              int64_t* expert_offsets, int32_t* group_counts, int64_t* group_offsets,
+              int32_t* row_of_pair, int32_t* pair_of_row,
+              void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------- dispatch */
+
+/* Permute (dispatch copy): xp[row_of_pair[t*k+j], :] = x[t, :].
+ *   x [T, d] dtype; row_of_pair [T*k] int32; xp [T*k, d] dtype output.
+ * Errors: INVALID_ARG, UNSUPPORTED (d not a multiple of 8). */
+MOE_API int moe_permute(const void* x, int dtype, int64_t T, int d, int k,
+                const int32_t* row_of_pair, void* xp, cudaStream_t stream);
+
+/* Workspace of moe_grouped_ffn_fwd, in bytes. */
+MOE_API size_t moe_grouped_ffn_fwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype);
+
+/* Grouped SwiGLU expert FFN, forward (grouped expert compute,
+ * leap-finetune PR #26 Summary; grouped-GEMM, ART issue #917). Rows
+ * [expert_offsets[e], expert_offsets[e+1]) of xp go through expert e:
+ *   h1 = xp Wg_e^T, h2 = xp Wu_e^T, a = silu(h1) * h2, yp = a Wd_e^T.
+ * The offsets are read on the device: an expert with no rows costs nothing
+ * and no host synchronisation is needed.
+ *   xp [rows, d]; Wg, Wu [E, f, d]; Wd [E, d, f]   dtype inputs
+ *   expert_offsets [E+1] int64 (from moe_route), expert_offsets[E] == rows
+ *   h1, h2, a [rows, f]; yp [rows, d]              dtype outputs
+ *     (h1, h2 and a are saved for the backward)
+ * Errors: INVALID_ARG; UNSUPPORTED (bf16 needs d and f multiples of 64,
+ * fp32 needs multiples of 4; E > MOE_MAX_EXPERTS); WORKSPACE. */
+MOE_API int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,
+                        int dtype, const int64_t* expert_offsets, int64_t rows, int E,
+                        int d, int f, void* h1, void* h2, void* a, void* yp,
+                        void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Unpermute and weighted combine (full source-order outputs, ART issue
+ * #917 Desired behavior):
+ *   Y[t, :] = sum_{j<k} topk_w[t,j] * yp[row_of_pair[t*k+j], :]
+ * summed in fp32 with j ascending, rounded once to dtype.
+ *   yp [T*k, d] dtype; topk_w [T, k] fp32; row_of_pair [T*k]; Y [T, d] dtype.
+ * Errors: INVALID_ARG, UNSUPPORTED (d not a multiple of 8). */
+MOE_API int moe_unpermute_combine(const void* yp, const float* topk_w, const int32_t* row_of_pair,
+                          int dtype, int64_t T, int d, int k, void* Y, cudaStream_t stream);
+
+/* --------------------------------------------------------- backward */
+
+/* Combine backward:
+ *   dyp[row_of_pair[t*k+j], :] = topk_w[t,j] * dY[t, :]
+ *   dg[t, j] = sum_i dY[t,i] * yp[row_of_pair[t*k+j], i]   (fp32)
+ *   dY [T, d] dtype; yp [T*k, d] dtype; dyp [T*k, d] dtype; dg [T, k] fp32. */
+MOE_API int moe_unpermute_combine_bwd(const void* dY, const void* yp, const float* topk_w,
+                              const int32_t* row_of_pair, int dtype, int64_t T, int d, int k,
+                              void* dyp, float* dg, cudaStream_t stream);
+
+/* Route backward through the softmax over the selected logits:
+ *   dlogits[t, S_j] = g_j * (dg_j - sum_m g_m dg_m), and 0 for every expert
+ *   not selected by token t.
+ *   dg, topk_w [T, k] fp32; topk_idx [T, k] int32; dlogits [T, E] fp32 output. */
+MOE_API int moe_route_bwd(const float* dg, const float* topk_w, const int32_t* topk_idx,
+                  int64_t T, int E, int k, float* dlogits, cudaStream_t stream);
+
+/* Workspace of moe_grouped_ffn_bwd, in bytes (holds dh1 and dh2). */
+MOE_API size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype);
+
+/* Grouped SwiGLU expert FFN, backward. Per expert e over its rows:
+ *   da  = dyp Wd_e;  dh1 = da * h2 * silu'(h1);  dh2 = da * silu(h1)
+ *   dxp = dh1 Wg_e + dh2 Wu_e                           (overwritten)
+ *   dWg_e += dh1^T xp;  dWu_e += dh2^T xp;  dWd_e += dyp^T a   (fp32, +=)
+ * with silu'(u) = s (1 + u (1 - s)), s = sigmoid(u). An expert with no rows
+ * leaves its gradients untouched.
+ *   xp, dyp [rows, d]; h1, h2, a [rows, f]; Wg, Wu [E, f, d]; Wd [E, d, f]
+ *   dxp [rows, d] dtype output; dWg, dWu [E, f, d], dWd [E, d, f] fp32 (+=).
+ * Errors: as moe_grouped_ffn_fwd. */
+MOE_API int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,
+                        const void* h1, const void* h2, const void* a, const void* dyp,
+                        int dtype, const int64_t* expert_offsets, int64_t rows, int E, int d,
+                        int f, void* dxp, float* dWg, float* dWu, float* dWd,
+                        void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Permute backward, with the router's input gradient folded in:
+ *   dX[t, :] = sum_{j<k} dxp[row_of_pair[t*k+j], :]
+ *            + sum_{j<k} dlogits[t, S_j] * Wr[S_j, :]      (if dlogits != NULL)
+ * summed in fp32 (j ascending), rounded once to dtype; dX is overwritten.
+ * The router term reads only the k selected columns of dlogits: it equals
+ * dlogits[t,:] Wr when dlogits is zero off the selection, which
+ * moe_route_bwd guarantees.
+ *   dxp [T*k, d] dtype; row_of_pair [T*k]; dlogits [T, E] fp32 or NULL;
+ *   Wr [E, d] dtype (ignored if dlogits is NULL); topk_idx [T, k];
+ *   dX [T, d] dtype output. */
+MOE_API int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dlogits,
+                    const void* Wr, const int32_t* topk_idx, int dtype, int64_t T, int d,
+                    int E, int k, void* dX, cudaStream_t stream);
+
+/* Workspace of moe_router_bwd, in bytes. */
+MOE_API size_t moe_router_bwd_workspace_bytes(int64_t T, int d, int E);
+
+/* Router weight gradients (accumulated, fp32, deterministic order):
+ *   dWr[e, :] += sum_t dlogits[t, e] x[t, :];   db[e] += sum_t dlogits[t, e]
+ *   x [T, d] dtype; dlogits [T, E] fp32; dWr [E, d] fp32; db [E] fp32 (may be
+ *   NULL). */
+MOE_API int moe_router_bwd(const void* x, const float* dlogits, int dtype, int64_t T, int d, int E,
+                   float* dWr, float* db, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

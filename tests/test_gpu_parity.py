@@ -1,0 +1,226 @@
+"""GPU parity: every step of the layer, through the C ABI, against the oracle.
+
+Integer results (top-k indices, counts, offsets, groups, permutation) and the
+fp32 router logits must match bit for bit; float results must be within the
+normwise tolerance of tests/parity.py. Sizes span several 128-row tiles and
+ragged tails; edge cases cover T = 0 and T = 1, starved experts, ties and
+non-finite logits.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from grouped_expert_ffn_top_b200 import native as N
+from grouped_expert_ffn_top_b200 import workloads
+from grouped_expert_ffn_top_b200.layer import MoELayer
+from parity import TOL, assert_close, check_routing_bitexact, oracle_routing, rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    N.lib()
+
+
+# ------------------------------------------------------------------ routing
+
+@pytest.mark.parametrize("T,E,k,G", [(1, 4, 2, 2), (255, 8, 2, 1), (256, 8, 2, 2), (257, 64, 8, 4),
+                                     (5000, 64, 8, 4), (3000, 16, 2, 1), (1000, 128, 4, 8),
+                                     (600, 1024, 8, 16), (100, 33, 32, 1), (70, 40, 1, 5)])
+def test_route_bitexact_on_tied_logits(T, E, k, G):
+    z = workloads.make_logits(T, E, seed=T * 7 + E)
+    out = N.moe_route(z.to(DEV), k, G)
+    idx, w, flags = oracle.route(z.double().numpy(), k)
+    lay = oracle.dispatch_layout(idx, E, G)
+    check_routing_bitexact(out, None, dict(idx=idx, w=w, **lay), check_logits=False)
+
+
+def test_route_nonfinite_logits_raise_the_device_flag():
+    z = workloads.make_logits(300, 16, seed=5, specials=True)
+    z[7, :] = -float("inf")
+    z[9, 3] = float("nan")
+    ws = N._ws(N.moe_route_workspace_bytes(300, 16), DEV)
+    out = N.moe_route(z.to(DEV), 4, 1, ws=ws)
+    assert N.moe_get_error(ws) & N.MOE_DEVERR_NONFINITE_LOGIT
+    assert N.moe_get_error(ws) == 0  # cleared by the read
+    idx, w, flags = oracle.route(z.double().numpy(), 4)
+    assert flags & oracle.FLAG_NONFINITE
+    assert np.array_equal(to_np(out["topk_idx"]), idx)
+    assert np.array_equal(to_np(out["topk_w"])[7], np.full(4, 0.25, np.float32))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("T,d,E", [(1, 64, 4), (300, 264, 8), (129, 1024, 16), (1000, 512, 64),
+                                   (77, 128, 100)])
+def test_router_logits_bitexact(dtype, T, d, E):
+    w = workloads.custom("l", T, d, E, 1, 64, dtype="bf16" if dtype == torch.bfloat16 else "f32")
+    p = workloads.make_params(w, device=DEV, seed=T + d)
+    x = workloads.make_batch(w, device=DEV, seed=E)["x"]
+    z = N.moe_router_logits(x, p["Wr"], p["b"])
+    ref = oracle.router_logits_f32(to_np(x), to_np(p["Wr"]), to_np(p["b"]))
+    assert np.array_equal(to_np(z), ref)
+
+
+# --------------------------------------------------------- whole layer
+
+LAYER_CASES = [
+    # name, T, d, E, k, f, dtype, G, starve_last
+    ("bf16_two_tiles", 700, 256, 8, 2, 384, "bf16", 2, True),
+    ("bf16_ragged", 333, 192, 5, 3, 320, "bf16", 1, False),
+    ("bf16_single_token", 1, 128, 4, 2, 128, "bf16", 2, False),
+    ("bf16_long_k", 2048, 512, 4, 1, 256, "bf16", 1, True),
+    ("bf16_f_not_256", 520, 320, 6, 2, 448, "bf16", 3, True),
+    ("f32_tiny", 256, 64, 4, 2, 128, "f32", 2, True),
+    ("f32_odd", 100, 48, 3, 2, 20, "f32", 1, False),
+]
+
+
+def _layer_case(T, d, E, k, f, dtype, G, starve, seed=0):
+    w = workloads.custom("case", T, d, E, k, f, dtype=dtype, bias=("normal", 0.5), ep_groups=G)
+    p = workloads.make_params(w, device=DEV, seed=seed)
+    if starve:
+        p["b"][E - 1] = -1.0e4
+    bt = workloads.make_batch(w, device=DEV, seed=seed)
+    return w, p, bt
+
+
+def _np_params(p):
+    return {n: to_np(v).astype(np.float64) for n, v in p.items()}
+
+
+@pytest.mark.parametrize("case", LAYER_CASES, ids=[c[0] for c in LAYER_CASES])
+def test_layer_forward_backward_matches_oracle(case):
+    _, T, d, E, k, f, dtype, G, starve = case
+    w, p, bt = _layer_case(T, d, E, k, f, dtype, G, starve)
+    tol = TOL[w.torch_dtype()]
+    layer = MoELayer(p, k, G, max_tokens=T)
+    Y = layer.forward(bt["x"])
+    dX = layer.backward(bt["dY"])
+    torch.cuda.synchronize()
+    assert layer.device_errors() == 0
+
+    ref_route = oracle_routing(bt["x"], p["Wr"], p["b"], k, G)
+    check_routing_bitexact(layer.r, layer.v["logits"], ref_route)
+    if starve:
+        assert ref_route["counts"][E - 1] == 0
+
+    P = _np_params(p)
+    x64 = to_np(bt["x"]).astype(np.float64)
+    dY64 = to_np(bt["dY"]).astype(np.float64)
+    fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k, G)
+    assert np.array_equal(fw["idx"], ref_route["idx"])
+    bw = oracle.layer_backward(fw, x64, dY64, P["Wr"], P["Wg"], P["Wu"], P["Wd"], k)
+
+    v = layer.v
+    assert np.array_equal(to_np(v["xp"]), fw["xp"]), "permute must copy rows exactly"
+    for n in ("h1", "h2", "a", "yp"):
+        assert_close(n, v[n], fw[n], tol)
+    assert_close("Y", Y, fw["Y"], tol)
+    assert_close("dyp", v["dyp"], bw["dyp"], tol)
+    assert_close("dg", v["dg"], bw["dg"], tol)
+    assert_close("dlogits", v["dlogits"], bw["dz"], tol)
+    assert_close("dxp", v["dxp"], bw["dxp"], tol)
+    assert_close("dX", dX, bw["dX"], tol)
+    g = layer.grads
+    for n in ("dWg", "dWu", "dWd", "dWr", "db"):
+        assert_close(n, g[n], bw[n], tol)
+    if starve:
+        for n in ("dWg", "dWu", "dWd"):
+            assert not g[n][E - 1].any(), f"{n} of the starved expert must stay exactly zero"
+
+
+def test_microbatches_accumulate_like_one_batch():
+    """Uneven microbatches (including T=0 and T=1) accumulate dW in fp32."""
+    d, E, k, f = 128, 4, 2, 192
+    w = workloads.custom("mb", [200, 0, 1, 77], d, E, k, f, bias=("normal", 0.5))
+    p = workloads.make_params(w, device=DEV, seed=3)
+    layer = MoELayer(p, k, 1, max_tokens=200)
+    P = _np_params(p)
+    acc = None
+    for mb in range(4):
+        bt = workloads.make_batch(w, mb=mb, device=DEV, seed=3)
+        Y = layer.forward(bt["x"])
+        dX = layer.backward(bt["dY"])
+        x64 = to_np(bt["x"]).astype(np.float64)
+        fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k)
+        bw = oracle.layer_backward(fw, x64, to_np(bt["dY"]).astype(np.float64), P["Wr"], P["Wg"],
+                                   P["Wu"], P["Wd"], k, acc=acc)
+        acc = {n: bw[n] for n in ("dWg", "dWu", "dWd", "dWr", "db")}
+        assert Y.shape == (w.T[mb], d) and dX.shape == (w.T[mb], d)
+        if w.T[mb]:
+            assert_close("Y", Y, fw["Y"], TOL[torch.bfloat16])
+            assert_close("dX", dX, bw["dX"], TOL[torch.bfloat16])
+    torch.cuda.synchronize()
+    for n, ref in acc.items():
+        assert_close(n, layer.grads[n], ref, TOL[torch.bfloat16])
+
+
+def test_empty_microbatch_changes_nothing():
+    d, E, k, f = 128, 4, 2, 128
+    w = workloads.custom("e", [64], d, E, k, f)
+    p = workloads.make_params(w, device=DEV)
+    layer = MoELayer(p, k, 2, max_tokens=64)
+    bt = workloads.make_batch(w, device=DEV)
+    layer.forward(bt["x"])
+    layer.backward(bt["dY"])
+    torch.cuda.synchronize()
+    before = {n: t.clone() for n, t in layer.grads.items()}
+    x0 = torch.empty((0, d), dtype=torch.bfloat16, device=DEV)
+    Y = layer.forward(x0)
+    dX = layer.backward(x0)
+    torch.cuda.synchronize()
+    assert Y.shape == (0, d) and dX.shape == (0, d)
+    for n in before:
+        assert torch.equal(before[n], layer.grads[n])
+
+
+def test_all_tokens_on_one_expert():
+    """Extreme skew: one expert takes every token, the others none."""
+    T, d, E, k, f = 1000, 128, 8, 1, 128
+    w = workloads.custom("skew", T, d, E, k, f, bias="zero")
+    p = workloads.make_params(w, device=DEV, seed=11)
+    p["b"][:] = -1.0e4
+    p["b"][5] = 0.0
+    bt = workloads.make_batch(w, device=DEV, seed=11)
+    layer = MoELayer(p, k, 1, max_tokens=T)
+    Y = layer.forward(bt["x"])
+    layer.backward(bt["dY"])
+    torch.cuda.synchronize()
+    counts = to_np(layer.r["counts"])
+    assert counts[5] == T and counts.sum() == T
+    P = _np_params(p)
+    x64 = to_np(bt["x"]).astype(np.float64)
+    fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k)
+    bw = oracle.layer_backward(fw, x64, to_np(bt["dY"]).astype(np.float64), P["Wr"], P["Wg"], P["Wu"],
+                               P["Wd"], k)
+    assert_close("Y", Y, fw["Y"], 2e-2)
+    for n in ("dWg", "dWu", "dWd"):
+        assert_close(n, layer.grads[n], bw[n], 2e-2)
+
+
+# ------------------------------------------------------- argument errors
+
+def test_rejected_calls_report_errors_and_launch_nothing():
+    z = torch.zeros((4, 8), device=DEV)
+    with pytest.raises(N.MoeError) as ei:
+        N.moe_route(z, 9)  # k > E
+    assert ei.value.code == N.MOE_ERR_INVALID_ARG
+    with pytest.raises(N.MoeError) as ei:
+        N.moe_route(z, 2, ep_groups=3)  # E % groups != 0
+    assert ei.value.code == N.MOE_ERR_UNSUPPORTED
+    with pytest.raises(N.MoeError) as ei:
+        N.moe_route(z, 2, ws=torch.zeros(16, dtype=torch.uint8, device=DEV))
+    assert ei.value.code == N.MOE_ERR_WORKSPACE
+    xp = torch.zeros((8, 100), dtype=torch.bfloat16, device=DEV)  # d not a multiple of 64
+    Wg = torch.zeros((2, 128, 100), dtype=torch.bfloat16, device=DEV)
+    Wd = torch.zeros((2, 100, 128), dtype=torch.bfloat16, device=DEV)
+    off = torch.tensor([0, 4, 8], dtype=torch.int64, device=DEV)
+    with pytest.raises(N.MoeError) as ei:
+        N.moe_grouped_ffn_fwd(xp, Wg, Wg, Wd, off)
+    assert ei.value.code == N.MOE_ERR_UNSUPPORTED
