@@ -2,6 +2,7 @@
 // Every check runs before anything is launched, so a rejected call changes
 // nothing on the device.
 #include <stdarg.h>
+#include <atomic>
 #include <stdio.h>
 
 #include "common.cuh"
@@ -10,6 +11,15 @@
 namespace {
 
 thread_local char g_msg[512] = "";
+std::atomic<int64_t> g_launches{0};
+
+void counted(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Adds the launches of a call that succeeded; passes the status through.
+int launched(int rc, int n) {
+  if (rc == MOE_OK) counted(n);
+  return rc;
+}
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -67,6 +77,8 @@ const char* moe_last_error(void) { return g_msg; }
 
 int moe_version(void) { return 1; }
 
+int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
 int moe_get_error(void* ws, cudaStream_t stream) {
   if (!ws) return fail(MOE_ERR_INVALID_ARG, "moe_get_error: null workspace");
   unsigned h = 0;
@@ -88,8 +100,8 @@ int moe_router_logits(const void* x, const void* Wr, const float* b, int dtype, 
   if (d % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "moe_router_logits: d=%d not a multiple of 8", d);
   if (T == 0) return MOE_OK;
   if (!x || !Wr || !logits) return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: null pointer");
-  return cuda_status(moe::launch_router_logits(x, Wr, b, dtype, T, d, E, logits, stream),
-                     "moe_router_logits");
+  return launched(cuda_status(moe::launch_router_logits(x, Wr, b, dtype, T, d, E, logits, stream),
+                              "moe_router_logits"), 1);
 }
 
 size_t moe_route_workspace_bytes(int64_t T, int E) {
@@ -131,7 +143,7 @@ int moe_route(const float* logits, int64_t T, int E, int k, int ep_groups, int32
   return cuda_status(moe::launch_route(logits, T, E, k, ep_groups, topk_idx, topk_w, expert_counts,
                                        expert_offsets, group_counts, group_offsets, row_of_pair,
                                        pair_of_row, block_counts, block_base, err, stream),
-                     "moe_route");
+                     "moe_route") == MOE_OK ? launched(MOE_OK, 3) : MOE_ERR_CUDA;
 }
 
 int moe_route_bwd(const float* dg, const float* topk_w, const int32_t* topk_idx, int64_t T, int E,
@@ -141,8 +153,8 @@ int moe_route_bwd(const float* dg, const float* topk_w, const int32_t* topk_idx,
   if (T == 0) return MOE_OK;
   if (!dg || !topk_w || !topk_idx || !dlogits)
     return fail(MOE_ERR_INVALID_ARG, "moe_route_bwd: null pointer");
-  return cuda_status(moe::launch_route_bwd(dg, topk_w, topk_idx, T, E, k, dlogits, stream),
-                     "moe_route_bwd");
+  return launched(cuda_status(moe::launch_route_bwd(dg, topk_w, topk_idx, T, E, k, dlogits, stream),
+                              "moe_route_bwd"), 1);
 }
 
 // ----------------------------------------------------------------- dispatch
@@ -154,7 +166,8 @@ int moe_permute(const void* x, int dtype, int64_t T, int d, int k, const int32_t
   if (T == 0) return MOE_OK;
   if (!x || !row_of_pair || !xp) return fail(MOE_ERR_INVALID_ARG, "moe_permute: null pointer");
   if (!aligned16(x) || !aligned16(xp)) return fail(MOE_ERR_INVALID_ARG, "moe_permute: 16-byte alignment");
-  return cuda_status(moe::launch_permute(x, dtype, T, d, k, row_of_pair, xp, stream), "moe_permute");
+  return launched(cuda_status(moe::launch_permute(x, dtype, T, d, k, row_of_pair, xp, stream),
+                              "moe_permute"), 1);
 }
 
 int moe_unpermute_combine(const void* yp, const float* topk_w, const int32_t* row_of_pair,
@@ -166,8 +179,8 @@ int moe_unpermute_combine(const void* yp, const float* topk_w, const int32_t* ro
     return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine: null pointer");
   if (!aligned16(yp) || !aligned16(Y))
     return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine: 16-byte alignment");
-  return cuda_status(moe::launch_combine(yp, topk_w, row_of_pair, dtype, T, d, k, Y, stream),
-                     "moe_unpermute_combine");
+  return launched(cuda_status(moe::launch_combine(yp, topk_w, row_of_pair, dtype, T, d, k, Y, stream),
+                              "moe_unpermute_combine"), 1);
 }
 
 int moe_unpermute_combine_bwd(const void* dY, const void* yp, const float* topk_w,
@@ -180,9 +193,9 @@ int moe_unpermute_combine_bwd(const void* dY, const void* yp, const float* topk_
     return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine_bwd: null pointer");
   if (!aligned16(dY) || !aligned16(yp) || !aligned16(dyp))
     return fail(MOE_ERR_INVALID_ARG, "moe_unpermute_combine_bwd: 16-byte alignment");
-  return cuda_status(
-      moe::launch_combine_bwd(dY, yp, topk_w, row_of_pair, dtype, T, d, k, dyp, dg, stream),
-      "moe_unpermute_combine_bwd");
+  return launched(cuda_status(moe::launch_combine_bwd(dY, yp, topk_w, row_of_pair, dtype, T, d, k,
+                                                      dyp, dg, stream),
+                              "moe_unpermute_combine_bwd"), 1);
 }
 
 int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dlogits,
@@ -198,7 +211,7 @@ int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dl
     return fail(MOE_ERR_INVALID_ARG, "moe_permute_bwd: 16-byte alignment");
   return cuda_status(moe::launch_permute_bwd(dxp, row_of_pair, dlogits, Wr, topk_idx, dtype, T, d,
                                              E, k, dX, stream),
-                     "moe_permute_bwd");
+                     "moe_permute_bwd") == MOE_OK ? launched(MOE_OK, 1) : MOE_ERR_CUDA;
 }
 
 size_t moe_router_bwd_workspace_bytes(int64_t T, int d, int E) {
@@ -218,8 +231,9 @@ int moe_router_bwd(const void* x, const float* dlogits, int dtype, int64_t T, in
     return fail(MOE_ERR_WORKSPACE, "moe_router_bwd: workspace needs %zu bytes",
                 moe_router_bwd_workspace_bytes(T, d, E));
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + moe::kWsHeader);
-  return cuda_status(moe::launch_router_bwd(x, dlogits, dtype, T, d, E, dWr, db, partial, stream),
-                     "moe_router_bwd");
+  return launched(cuda_status(moe::launch_router_bwd(x, dlogits, dtype, T, d, E, dWr, db, partial,
+                                                      stream),
+                              "moe_router_bwd"), 2);
 }
 
 // ------------------------------------------------------------ grouped FFN
@@ -247,7 +261,7 @@ int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const vo
                        static_cast<unsigned*>(ws)};
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_fwd_bf16(args, stream)
                                     : moe::launch_ffn_fwd_f32(args, stream);
-  return cuda_status(e, "moe_grouped_ffn_fwd");
+  return launched(cuda_status(e, "moe_grouped_ffn_fwd"), 2);
 }
 
 size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype) {
@@ -279,9 +293,55 @@ int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const vo
   moe::FfnBwdArgs args{xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, rows, E, d, f, dxp,
                        dWg, dWu, dWd, base + moe::kWsHeader, base + moe::kWsHeader + h,
                        static_cast<unsigned*>(ws)};
-  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_bwd_bf16(args, stream)
-                                    : moe::launch_ffn_bwd_f32(args, stream);
-  return cuda_status(e, "moe_grouped_ffn_bwd");
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
+                                    : moe::launch_ffn_dgrad_f32(args, stream);
+  if (e == cudaSuccess) {
+    counted(2);
+    e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
+                          : moe::launch_ffn_wgrad_f32(args, stream);
+  }
+  return launched(cuda_status(e, "moe_grouped_ffn_bwd"), 1);
+}
+
+int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const void* h1,
+                          const void* h2, const void* dyp, int dtype, const int64_t* expert_offsets,
+                          int64_t rows, int E, int d, int f, void* dh1, void* dh2, void* dxp,
+                          void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_ffn("moe_grouped_ffn_dgrad", dtype, rows, E, d, f);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!Wg || !Wu || !Wd || !h1 || !h2 || !dyp || !expert_offsets || !dh1 || !dh2 || !dxp || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_dgrad: null pointer");
+  const void* ptrs[] = {Wg, Wu, Wd, h1, h2, dyp, dh1, dh2, dxp, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_dgrad: 16-byte alignment");
+  if (ws_bytes < moe::kWsHeader) return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_dgrad: workspace");
+  moe::FfnBwdArgs args{nullptr, Wg, Wu, Wd, h1, h2, nullptr, dyp, expert_offsets, rows, E, d, f,
+                       dxp, nullptr, nullptr, nullptr, dh1, dh2, static_cast<unsigned*>(ws)};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
+                                    : moe::launch_ffn_dgrad_f32(args, stream);
+  return launched(cuda_status(e, "moe_grouped_ffn_dgrad"), 2);
+}
+
+int moe_grouped_ffn_wgrad(const void* xp, const void* a, const void* dyp, const void* dh1,
+                          const void* dh2, int dtype, const int64_t* expert_offsets, int64_t rows,
+                          int E, int d, int f, float* dWg, float* dWu, float* dWd, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_ffn("moe_grouped_ffn_wgrad", dtype, rows, E, d, f);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!xp || !a || !dyp || !dh1 || !dh2 || !expert_offsets || !dWg || !dWu || !dWd || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: null pointer");
+  const void* ptrs[] = {xp, a, dyp, dh1, dh2, dWg, dWu, dWd, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: 16-byte alignment");
+  if (ws_bytes < moe::kWsHeader) return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_wgrad: workspace");
+  moe::FfnBwdArgs args{xp, nullptr, nullptr, nullptr, nullptr, nullptr, a, dyp, expert_offsets,
+                       rows, E, d, f, nullptr, dWg, dWu, dWd, const_cast<void*>(dh1),
+                       const_cast<void*>(dh2), static_cast<unsigned*>(ws)};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
+                                    : moe::launch_ffn_wgrad_f32(args, stream);
+  return launched(cuda_status(e, "moe_grouped_ffn_wgrad"), 1);
 }
 
 }  // extern "C"

@@ -644,15 +644,20 @@ cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   return launch<kFwdDown, 256>(m2, p, s);
 }
 
-cudaError_t launch_ffn_bwd_bf16(const FfnBwdArgs& a, cudaStream_t s) {
-  using namespace gg;
-  const uint64_t rows = static_cast<uint64_t>(a.rows), E = a.E, d = a.d, f = a.f;
-  Params p{};
+static gg::Params bwd_params(const FfnBwdArgs& a) {
+  gg::Params p{};
   p.offsets = a.offsets;
   p.E = a.E;
   p.d = a.d;
   p.f = a.f;
   p.err = a.err;
+  return p;
+}
+
+cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
+  using namespace gg;
+  const uint64_t rows = static_cast<uint64_t>(a.rows), E = a.E, d = a.d, f = a.f;
+  Params p = bwd_params(a);
   // 1. da = dyp Wd_e, SwiGLU backward in the epilogue -> dh1, dh2
   Maps m1{};
   if (!make_map(&m1.a0, a.dyp, d, rows, d, 64, 128) || !make_map(&m1.b0, a.Wd, f, E * d, f, 64, 64))
@@ -672,15 +677,18 @@ cudaError_t launch_ffn_bwd_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.i0 = p.i1 = nullptr;
   p.o0 = static_cast<bf16*>(a.dxp);
   p.o1 = nullptr;
-  e = launch<kBwdDgradGateUp, 256>(m2, p, s);
-  if (e != cudaSuccess) return e;
-  // 3. weight gradients, accumulated in fp32
+  return launch<kBwdDgradGateUp, 256>(m2, p, s);
+}
+
+cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
+  using namespace gg;
+  const uint64_t rows = static_cast<uint64_t>(a.rows), d = a.d, f = a.f;
+  Params p = bwd_params(a);
   Maps m3{};
   if (!make_map(&m3.a0, a.dh1, f, rows, f, 64, 64) || !make_map(&m3.a1, a.dh2, f, rows, f, 64, 64) ||
       !make_map(&m3.a2, a.a, f, rows, f, 64, 64) || !make_map(&m3.b0, a.xp, d, rows, d, 64, 64) ||
       !make_map(&m3.b1, a.dyp, d, rows, d, 64, 64))
     return cudaErrorInvalidValue;
-  p.o0 = nullptr;
   p.w0 = a.dWg;
   p.w1 = a.dWu;
   p.w2 = a.dWd;

@@ -147,7 +147,7 @@ cudaError_t launch_ffn_fwd_f32(const FfnFwdArgs& x, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_ffn_bwd_f32(const FfnBwdArgs& x, cudaStream_t s) {
+cudaError_t launch_ffn_dgrad_f32(const FfnBwdArgs& x, cudaStream_t s) {
   float* dh1 = static_cast<float*>(x.dh1);
   float* dh2 = static_cast<float*>(x.dh2);
   simt_dgrad_down_kernel<<<blocks_for(x.rows * x.f), 256, 0, s>>>(
@@ -159,8 +159,12 @@ cudaError_t launch_ffn_bwd_f32(const FfnBwdArgs& x, cudaStream_t s) {
   simt_dgrad_gateup_kernel<<<blocks_for(x.rows * x.d), 256, 0, s>>>(
       dh1, dh2, static_cast<const float*>(x.Wg), static_cast<const float*>(x.Wu), x.offsets,
       x.rows, x.E, x.d, x.f, static_cast<float*>(x.dxp));
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ffn_wgrad_f32(const FfnBwdArgs& x, cudaStream_t s) {
+  const float* dh1 = static_cast<const float*>(x.dh1);
+  const float* dh2 = static_cast<const float*>(x.dh2);
   simt_wgrad_kernel<<<blocks_for(static_cast<int64_t>(x.E) * x.f * x.d), 256, 0, s>>>(
       static_cast<const float*>(x.xp), static_cast<const float*>(x.dyp),
       static_cast<const float*>(x.a), dh1, dh2, x.offsets, x.E, x.d, x.f, x.dWg, x.dWu, x.dWd);

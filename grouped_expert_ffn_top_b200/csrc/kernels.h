@@ -54,13 +54,15 @@ struct FfnBwdArgs {
   int E, d, f;
   void* dxp;
   float *dWg, *dWu, *dWd;
-  void *dh1, *dh2;  // scratch [rows, f]
+  void *dh1, *dh2;  // [rows, f]: written by dgrad, read by wgrad
   unsigned* err;
 };
 
 cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s);
-cudaError_t launch_ffn_bwd_bf16(const FfnBwdArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 2 launches
+cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 1 launch
 cudaError_t launch_ffn_fwd_f32(const FfnFwdArgs& a, cudaStream_t s);
-cudaError_t launch_ffn_bwd_f32(const FfnBwdArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_dgrad_f32(const FfnBwdArgs& a, cudaStream_t s);   // 2 launches
+cudaError_t launch_ffn_wgrad_f32(const FfnBwdArgs& a, cudaStream_t s);   // 1 launch
 
 }  // namespace moe

@@ -87,6 +87,11 @@ MOE_API const char* moe_last_error(void);
 /* Library ABI version (increments on any signature change). */
 MOE_API int moe_version(void);
 
+/* Number of kernels this library has launched in the process so far (all
+ * devices, all threads). A diagnostic: differences around a region count the
+ * library's launches in it. */
+MOE_API int64_t moe_launch_count(void);
+
 /* Synchronises `stream`, returns the device error word accumulated in `ws`
  * by the calls that used it since the last moe_get_error (0 = no error), and
  * clears it. Returns MOE_ERR_CUDA (< 0) if the synchronisation fails. */
@@ -216,6 +221,25 @@ MOE_API int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, 
                         int dtype, const int64_t* expert_offsets, int64_t rows, int E, int d,
                         int f, void* dxp, float* dWg, float* dWu, float* dWd,
                         void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* The two halves of moe_grouped_ffn_bwd, for callers that keep dh1 / dh2
+ * themselves (and may schedule the weight gradient apart from the data
+ * gradient). Same arithmetic as moe_grouped_ffn_bwd.
+ * moe_grouped_ffn_dgrad: data gradients
+ *   dh1, dh2 [rows, f] dtype outputs (the SwiGLU backward of da = dyp Wd_e)
+ *   dxp [rows, d] dtype output (= dh1 Wg_e + dh2 Wu_e)
+ * moe_grouped_ffn_wgrad: weight gradients, accumulated in fp32
+ *   dWg_e += dh1^T xp; dWu_e += dh2^T xp; dWd_e += dyp^T a
+ * ws needs moe_grouped_ffn_fwd_workspace_bytes() bytes (its error word). */
+MOE_API int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const void* h1,
+                                  const void* h2, const void* dyp, int dtype,
+                                  const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
+                                  void* dh1, void* dh2, void* dxp, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream);
+MOE_API int moe_grouped_ffn_wgrad(const void* xp, const void* a, const void* dyp, const void* dh1,
+                                  const void* dh2, int dtype, const int64_t* expert_offsets,
+                                  int64_t rows, int E, int d, int f, float* dWg, float* dWu,
+                                  float* dWd, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Permute backward, with the router's input gradient folded in:
  *   dX[t, :] = sum_{j<k} dxp[row_of_pair[t*k+j], :]
