@@ -2,8 +2,9 @@
 
 Forward:  moe_router_logits -> moe_route -> moe_permute -> moe_grouped_ffn_fwd
           -> moe_unpermute_combine
-Backward: moe_unpermute_combine_bwd -> moe_route_bwd -> moe_grouped_ffn_bwd
-          -> moe_permute_bwd (with the router's input gradient) -> moe_router_bwd
+Backward: moe_unpermute_combine_bwd -> moe_route_bwd -> moe_grouped_ffn_dgrad
+          -> moe_grouped_ffn_wgrad -> moe_permute_bwd (with the router's input
+          gradient) -> moe_router_bwd
 
 The object owns device buffers sized for `max_tokens`, so a step allocates
 nothing; microbatches of any size up to that (0 included) reuse them. Weight
@@ -16,6 +17,18 @@ from typing import Dict, Optional
 import torch
 
 from . import native as N
+
+
+def _no_mark(name: str) -> None:
+    pass
+
+
+# Kernels each C call launches (bf16 and fp32 paths alike).
+LAUNCHES_PER_CALL = {
+    "router_logits": 1, "route": 3, "permute": 1, "grouped_ffn_fwd": 2, "unpermute_combine": 1,
+    "unpermute_combine_bwd": 1, "route_bwd": 1, "grouped_ffn_dgrad": 2, "grouped_ffn_wgrad": 1,
+    "permute_bwd": 1, "router_bwd": 2,
+}
 
 
 class MoELayer:
@@ -60,13 +73,15 @@ class MoELayer:
             "dg": torch.empty((T, k), dtype=f32, device=dev),
             "dlogits": torch.empty((T, E), dtype=f32, device=dev),
             "dxp": torch.empty((P, d), dtype=dt, device=dev),
+            "dh1": torch.empty((P, f), dtype=dt, device=dev),
+            "dh2": torch.empty((P, f), dtype=dt, device=dev),
             "dX": torch.empty((T, d), dtype=dt, device=dev),
         }
         self.route = N.route_outputs(T, E, k, self.G, dev)
         self.ws = {
             "route": N._ws(N.moe_route_workspace_bytes(T, E), dev),
             "ffn_fwd": N._ws(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt), dev),
-            "ffn_bwd": N._ws(N.moe_grouped_ffn_bwd_workspace_bytes(P, E, d, f, self.dt), dev),
+            "ffn_bwd": N._ws(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt), dev),
             "router_bwd": N._ws(N.moe_router_bwd_workspace_bytes(T, d, E), dev),
         }
         self.max_tokens = T
@@ -80,7 +95,7 @@ class MoELayer:
         b = self.buf
         r = self.route
         v = {n: b[n][:T] for n in ("logits", "Y", "dg", "dlogits", "dX")}
-        v.update({n: b[n][:P] for n in ("xp", "h1", "h2", "a", "yp", "dyp", "dxp")})
+        v.update({n: b[n][:P] for n in ("xp", "h1", "h2", "a", "yp", "dyp", "dxp", "dh1", "dh2")})
         ro = dict(r)
         for n in ("topk_idx", "topk_w"):
             ro[n] = r[n][:T]
@@ -88,7 +103,10 @@ class MoELayer:
             ro[n] = r[n][:P]
         return v, ro
 
-    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, stream=None, mark=None) -> torch.Tensor:
+        """Y = layer(x). `mark(name)`, if given, is called after each C call
+        (the benchmark records CUDA events there)."""
+        mark = mark or _no_mark
         T = x.shape[0]
         self.reserve(T)
         self.T = T
@@ -96,25 +114,39 @@ class MoELayer:
         v, r = self._views(T)
         self.v, self.r = v, r
         N.moe_router_logits(x, self.Wr, self.b, v["logits"], stream)
+        mark("router_logits")
         N.moe_route(v["logits"], self.k, self.G, r, self.ws["route"], stream)
+        mark("route")
         N.moe_permute(x, r["row_of_pair"], self.k, v["xp"], stream)
+        mark("permute")
         N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"],
                               {n: v[n] for n in ("h1", "h2", "a", "yp")}, self.ws["ffn_fwd"], stream)
+        mark("grouped_ffn_fwd")
         N.moe_unpermute_combine(v["yp"], r["topk_w"], r["row_of_pair"], v["Y"], stream)
+        mark("unpermute_combine")
         return v["Y"]
 
-    def backward(self, dY: torch.Tensor, stream=None) -> torch.Tensor:
+    def backward(self, dY: torch.Tensor, stream=None, mark=None) -> torch.Tensor:
+        """dX for upstream gradient dY of the last forward; dW += (fp32)."""
+        mark = mark or _no_mark
         T = self.T
         v, r = self.v, self.r
         g = self.grads
         N.moe_unpermute_combine_bwd(dY, v["yp"], r["topk_w"], r["row_of_pair"], v["dyp"], v["dg"], stream)
+        mark("unpermute_combine_bwd")
         N.moe_route_bwd(v["dg"], r["topk_w"], r["topk_idx"], self.E, v["dlogits"], stream)
-        N.moe_grouped_ffn_bwd(v["xp"], self.Wg, self.Wu, self.Wd, v["h1"], v["h2"], v["a"], v["dyp"],
-                              r["offsets"], g["dWg"], g["dWu"], g["dWd"], v["dxp"], self.ws["ffn_bwd"],
-                              stream)
+        mark("route_bwd")
+        N.moe_grouped_ffn_dgrad(self.Wg, self.Wu, self.Wd, v["h1"], v["h2"], v["dyp"], r["offsets"],
+                                v["dh1"], v["dh2"], v["dxp"], self.ws["ffn_bwd"], stream)
+        mark("grouped_ffn_dgrad")
+        N.moe_grouped_ffn_wgrad(v["xp"], v["a"], v["dyp"], v["dh1"], v["dh2"], r["offsets"], g["dWg"],
+                                g["dWu"], g["dWd"], self.ws["ffn_bwd"], stream)
+        mark("grouped_ffn_wgrad")
         N.moe_permute_bwd(v["dxp"], r["row_of_pair"], v["dlogits"], self.Wr, r["topk_idx"], T, self.k,
                           v["dX"], stream)
+        mark("permute_bwd")
         N.moe_router_bwd(self.x, v["dlogits"], g["dWr"], g["db"], self.ws["router_bwd"], stream)
+        mark("router_bwd")
         return v["dX"]
 
     def device_errors(self) -> int:

@@ -46,6 +46,7 @@ _sz = ctypes.c_size_t
 _SIGNATURES = {
     "moe_last_error": ([], ctypes.c_char_p),
     "moe_version": ([], _i),
+    "moe_launch_count": ([], _i64),
     "moe_get_error": ([_p, _p], _i),
     "moe_router_logits": ([_p, _p, _p, _i, _i64, _i, _i, _p, _p], _i),
     "moe_route_workspace_bytes": ([_i64, _i], _sz),
@@ -58,6 +59,8 @@ _SIGNATURES = {
     "moe_route_bwd": ([_p, _p, _p, _i64, _i, _i, _p, _p], _i),
     "moe_grouped_ffn_bwd_workspace_bytes": ([_i64, _i, _i, _i, _i], _sz),
     "moe_grouped_ffn_bwd": ([_p] * 8 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_grouped_ffn_dgrad": ([_p] * 6 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_grouped_ffn_wgrad": ([_p] * 5 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
     "moe_permute_bwd": ([_p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p], _i),
     "moe_router_bwd_workspace_bytes": ([_i64, _i, _i], _sz),
     "moe_router_bwd": ([_p, _p, _i, _i64, _i, _i, _p, _p, _p, _sz, _p], _i),
@@ -125,6 +128,10 @@ def moe_get_error(ws: torch.Tensor, stream=None) -> int:
     if rc < 0:
         _check(rc, "moe_get_error")
     return rc
+
+
+def moe_launch_count() -> int:
+    return lib().moe_launch_count()
 
 
 def moe_router_logits(x, Wr, b, logits=None, stream=None):
@@ -254,6 +261,27 @@ def moe_grouped_ffn_bwd(xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu
                                      _ptr(dxp), _ptr(dWg), _ptr(dWu), _ptr(dWd), _ptr(ws), ws.numel(),
                                      _stream(stream)), "moe_grouped_ffn_bwd")
     return dxp
+
+
+def moe_grouped_ffn_dgrad(Wg, Wu, Wd, h1, h2, dyp, expert_offsets, dh1, dh2, dxp, ws, stream=None):
+    _contig(Wg, Wu, Wd, h1, h2, dyp, expert_offsets, dh1, dh2, dxp)
+    rows, d = dyp.shape
+    E, f, _ = Wg.shape
+    _check(lib().moe_grouped_ffn_dgrad(_ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(h1), _ptr(h2), _ptr(dyp),
+                                       _dt(dyp), _ptr(expert_offsets), rows, E, d, f, _ptr(dh1),
+                                       _ptr(dh2), _ptr(dxp), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn_dgrad")
+    return dxp
+
+
+def moe_grouped_ffn_wgrad(xp, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd, ws, stream=None):
+    _contig(xp, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd)
+    rows, d = xp.shape
+    E, f, _ = dWg.shape
+    _check(lib().moe_grouped_ffn_wgrad(_ptr(xp), _ptr(a), _ptr(dyp), _ptr(dh1), _ptr(dh2), _dt(xp),
+                                       _ptr(expert_offsets), rows, E, d, f, _ptr(dWg), _ptr(dWu),
+                                       _ptr(dWd), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn_wgrad")
 
 
 def moe_permute_bwd(dxp, row_of_pair, dlogits, Wr, topk_idx, T: int, k: int, dX=None, stream=None):
