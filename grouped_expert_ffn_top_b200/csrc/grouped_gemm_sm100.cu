@@ -11,7 +11,7 @@
 //   kFwdDown        yp = a Wd_e^T
 //   kBwdDgradDown   da = dyp Wd_e, epilogue dh1 = da h2 silu'(h1), dh2 = da silu(h1)
 //   kBwdDgradGateUp dxp = [dh1 | dh2] [Wg_e ; Wu_e]          (K = 2f)
-//   kWgrad          dWg_e += dh1^T xp, dWu_e += dh2^T xp, dWd_e^T += a^T dyp
+//   kWgrad          dWg_e^T += xp^T dh1, dWu_e^T += xp^T dh2, dWd_e^T += a^T dyp
 // The first four have a ragged M (the expert's rows, tiles of 128; rows of a
 // tile past the expert's end are computed and discarded). kWgrad has a ragged
 // K (the expert's rows): in the last K block the rows past the expert's end
@@ -48,7 +48,7 @@ enum Kind : int {
 };
 
 struct Maps {
-  CUtensorMap a0, a1, a2, b0, b1;
+  CUtensorMap a0, a1, b0, b1, b2;
 };
 
 struct Params {
@@ -101,7 +101,7 @@ template <int KIND, int BN>
 __device__ __forceinline__ int tiles_of_expert(int cnt, int d, int f) {
   using Tr = Traits<KIND, BN>;
   if (cnt <= 0) return 0;
-  if (KIND == kWgrad) return 3 * ceil_div(f, BM) * ceil_div(d, BN);
+  if (KIND == kWgrad) return 2 * ceil_div(d, BM) * ceil_div(f, BN) + ceil_div(f, BM) * ceil_div(d, BN);
   const int n_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? f : d;
   return ceil_div(cnt, BM) * ceil_div(n_extent, Tr::NTILE);
 }
@@ -136,9 +136,19 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d,
   const int base = static_cast<int>(s.off[ti.e]);
   const int cnt = static_cast<int>(s.off[ti.e + 1] - s.off[ti.e]);
   if (KIND == kWgrad) {
-    const int nt = ceil_div(d, BN), mt = ceil_div(f, BM);
-    ti.prod = local / (mt * nt);
-    const int rem = local % (mt * nt);
+    // products 0, 1 (dWg, dWu): M over d, N over f; product 2 (dWd): M over f,
+    // N over d. M always runs along the output's contiguous dimension.
+    const int t01 = ceil_div(d, BM) * ceil_div(f, BN);
+    int rem, nt;
+    if (local < 2 * t01) {
+      ti.prod = local / t01;
+      rem = local % t01;
+      nt = ceil_div(f, BN);
+    } else {
+      ti.prod = 2;
+      rem = local - 2 * t01;
+      nt = ceil_div(d, BN);
+    }
     ti.m0 = (rem / nt) * BM;
     ti.n0 = (rem % nt) * BN;
     ti.row0 = base;
@@ -183,9 +193,9 @@ __device__ __forceinline__ void issue_loads(const Maps& m, const TileInfo& ti, i
 #pragma unroll
     for (int j = 0; j < BN / 64; ++j)
       tma_load_2d(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + 64 * j, ti.e * f + kk);
-  } else {  // kWgrad
-    const CUtensorMap* am = ti.prod == 0 ? &m.a0 : (ti.prod == 1 ? &m.a1 : &m.a2);
-    const CUtensorMap* bm = ti.prod == 2 ? &m.b1 : &m.b0;
+  } else {  // kWgrad: A = xp (dWg, dWu) or a (dWd); B = dh1, dh2 or dyp
+    const CUtensorMap* am = ti.prod == 2 ? &m.a1 : &m.a0;
+    const CUtensorMap* bm = ti.prod == 0 ? &m.b0 : (ti.prod == 1 ? &m.b1 : &m.b2);
     const int r = ti.row0 + k0;
     tma_load_2d(a_dst, am, bar, ti.m0, r);
     tma_load_2d(a_dst + 8192, am, bar, ti.m0 + 64, r);
@@ -221,6 +231,30 @@ __device__ __forceinline__ void store16_bf16(bf16* dst, const float* v) {
   uint4* p = reinterpret_cast<uint4*>(dst);
   p[0] = pack8_bf16(v);
   p[1] = pack8_bf16(v + 8);
+}
+
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// Work an epilogue thread can start before its accumulator is ready: pull
+// the h1 / h2 values the SwiGLU backward will read into L2.
+template <int KIND, int BN>
+__device__ __forceinline__ void epilogue_prefetch(const Params& p, const TileInfo& ti, int r) {
+  if (KIND == kBwdDgradDown) {
+    if (r < ti.rows) {
+      const int64_t off = (static_cast<int64_t>(ti.row0) + r) * p.f + ti.n0;
+      const int cols = min(BN, p.f - ti.n0);
+      for (int c = 0; c < cols; c += 64) {  // 64 bf16 = one 128-byte line
+        prefetch_l2(p.i0 + off + c);
+        prefetch_l2(p.i1 + off + c);
+      }
+    }
+  }
 }
 
 // Epilogue of one tile for this thread's accumulator row r.
@@ -291,41 +325,24 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
       }
     }
   } else {  // kWgrad
-    const int m = ti.m0 + r;  // f index
-    const bool valid = m < f;
-    if (ti.prod < 2) {
-      float* out = (ti.prod == 0 ? p.w0 : p.w1) + static_cast<int64_t>(ti.e) * f * d +
-                   static_cast<int64_t>(m) * d;
-      for (int c = 0; c < BN; c += 16) {
-        tmem_ld16(tacc + c, u);
-        tmem_ld_wait();
-        if (valid && ti.n0 + c < d) {
-          float4* o4 = reinterpret_cast<float4*>(out + ti.n0 + c);
+    // Accumulator row m, column n is element (n, m) of the [N, M] row-major
+    // output, so for each column the 32 lanes of a warp cover 32 consecutive
+    // floats: one coalesced 128-byte reduction per column. red.global.add is
+    // fire-and-forget (the add happens at L2), and each element receives
+    // exactly one add per call, so the result is deterministic.
+    const int M = ti.prod == 2 ? f : d;
+    const int Nn = ti.prod == 2 ? d : f;
+    const int m = ti.m0 + r;
+    const bool valid = m < M;
+    float* out = (ti.prod == 0 ? p.w0 : (ti.prod == 1 ? p.w1 : p.w2)) +
+                 static_cast<int64_t>(ti.e) * d * f + m;
+    for (int c = 0; c < BN; c += 16) {
+      tmem_ld16(tacc + c, u);
+      tmem_ld_wait();
+      if (valid && ti.n0 + c < Nn) {
+        float* q = out + static_cast<int64_t>(ti.n0 + c) * M;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float4 cur = o4[q];
-            cur.x += __uint_as_float(u[4 * q + 0]);
-            cur.y += __uint_as_float(u[4 * q + 1]);
-            cur.z += __uint_as_float(u[4 * q + 2]);
-            cur.w += __uint_as_float(u[4 * q + 3]);
-            o4[q] = cur;
-          }
-        }
-      }
-    } else {
-      // dWd_e is [d, f]: this row m is column m of it; lanes hold consecutive
-      // m, so each of the 16 updates is one coalesced 128-byte access per warp
-      float* out = p.w2 + static_cast<int64_t>(ti.e) * d * f + m;
-      for (int c = 0; c < BN; c += 16) {
-        tmem_ld16(tacc + c, u);
-        tmem_ld_wait();
-        if (valid && ti.n0 + c < d) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float* q = out + static_cast<int64_t>(ti.n0 + c + i) * f;
-            *q += __uint_as_float(u[i]);
-          }
-        }
+        for (int i = 0; i < 16; ++i) red_add_f32(q + static_cast<int64_t>(i) * M, __uint_as_float(u[i]));
       }
     }
   }
@@ -380,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&maps.b0);
     if (KIND == kBwdDgradGateUp || KIND == kWgrad) tma_prefetch_desc(&maps.a1);
     if (KIND == kFwdGateUp || KIND == kBwdDgradGateUp || KIND == kWgrad) tma_prefetch_desc(&maps.b1);
-    if (KIND == kWgrad) tma_prefetch_desc(&maps.a2);
+    if (KIND == kWgrad) tma_prefetch_desc(&maps.b2);
   }
   if (warp == 1) {
     tmem_alloc(s_tmem, kTmemCols);
@@ -544,6 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      epilogue_prefetch<KIND, BN>(p, ti, r);
       if (!wait_bounded(&tfull[acc], acc_phase, s_abort, kWaitLimit)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
@@ -685,9 +703,9 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   const uint64_t rows = static_cast<uint64_t>(a.rows), d = a.d, f = a.f;
   Params p = bwd_params(a);
   Maps m3{};
-  if (!make_map(&m3.a0, a.dh1, f, rows, f, 64, 64) || !make_map(&m3.a1, a.dh2, f, rows, f, 64, 64) ||
-      !make_map(&m3.a2, a.a, f, rows, f, 64, 64) || !make_map(&m3.b0, a.xp, d, rows, d, 64, 64) ||
-      !make_map(&m3.b1, a.dyp, d, rows, d, 64, 64))
+  if (!make_map(&m3.a0, a.xp, d, rows, d, 64, 64) || !make_map(&m3.a1, a.a, f, rows, f, 64, 64) ||
+      !make_map(&m3.b0, a.dh1, f, rows, f, 64, 64) || !make_map(&m3.b1, a.dh2, f, rows, f, 64, 64) ||
+      !make_map(&m3.b2, a.dyp, d, rows, d, 64, 64))
     return cudaErrorInvalidValue;
   p.w0 = a.dWg;
   p.w1 = a.dWu;
