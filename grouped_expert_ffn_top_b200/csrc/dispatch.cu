@@ -319,61 +319,118 @@ cudaError_t launch_permute_bwd(const void* dxp, const int32_t* row_of_pair, cons
 constexpr int kRbTile = 64;
 constexpr int kRbTok = 32;
 
+// Block: 64 experts x 64 columns of dWr, 64 threads, 8x8 register tile per
+// thread; tokens of the block's split in chunks of 32, staged with 16-byte
+// loads one chunk ahead (register double buffer).
 template <typename T>
-__global__ void __launch_bounds__(256) router_wgrad_partial_kernel(
+__global__ void __launch_bounds__(64) router_wgrad_partial_kernel(
     const T* __restrict__ x, const float* __restrict__ dz, int64_t Ttok, int d, int E,
     int64_t tok_per_split, float* __restrict__ partial, float* __restrict__ partial_db) {
+  constexpr int VE = Vec16<T>::N;
+  constexpr int XV = kRbTok * kRbTile / VE / 64;  // x vectors per thread per chunk
+  constexpr int ZV = kRbTok * kRbTile / 4 / 64;   // dz float4 per thread per chunk
   __shared__ __align__(16) float sz[kRbTok][kRbTile];
   __shared__ __align__(16) float sx[kRbTok][kRbTile];
   const int tid = threadIdx.x;
-  const int te = tid / 16, tc = tid % 16;
+  const int te = tid / 8, tc = tid % 8;
   const int c0 = blockIdx.x * kRbTile;
   const int split = blockIdx.y;
   const int e0 = blockIdx.z * kRbTile;
   const int64_t tb = split * tok_per_split;
   const int64_t tend = min(Ttok, tb + tok_per_split);
-  float acc[4][4];
+  const bool e_vec_ok = (E % 4 == 0);
+
+  Vec16<T> xr[XV];
+  float4 zr[ZV];
+  auto load_stage = [&](int64_t t0) {
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b) acc[a][b] = 0.0f;
-  float dbacc = 0.0f;
-  for (int64_t t0 = tb; t0 < tend; t0 += kRbTok) {
-    for (int i = tid; i < kRbTok * kRbTile; i += 256) {
-      const int tt = i / kRbTile, cc = i % kRbTile;
+    for (int j = 0; j < XV; ++j) {
+      const int vid = tid + 64 * j;
+      const int tt = vid / (kRbTile / VE), cv = vid % (kRbTile / VE);
       const int64_t t = t0 + tt;
-      const bool tv = t < tend;
-      sz[tt][cc] = (tv && e0 + cc < E) ? dz[t * E + e0 + cc] : 0.0f;
-      sx[tt][cc] = (tv && c0 + cc < d) ? to_f32(x[t * d + c0 + cc]) : 0.0f;
+      const int c = c0 + cv * VE;
+      if (t < tend && c < d) xr[j] = ld16_stream(x + t * d + c);
+      else xr[j].raw = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < ZV; ++j) {
+      const int vid = tid + 64 * j;
+      const int tt = vid / (kRbTile / 4), ev = vid % (kRbTile / 4);
+      const int64_t t = t0 + tt;
+      const int e = e0 + ev * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < tend) {
+        const float* src = dz + t * E + e;
+        if (e_vec_ok && e + 3 < E) {
+          v = __ldcs(reinterpret_cast<const float4*>(src));
+        } else {
+          if (e < E) v.x = src[0];
+          if (e + 1 < E) v.y = src[1];
+          if (e + 2 < E) v.z = src[2];
+          if (e + 3 < E) v.w = src[3];
+        }
+      }
+      zr[j] = v;
+    }
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.0f;
+  float dbacc = 0.0f;
+  if (tb < tend) load_stage(tb);
+  for (int64_t t0 = tb; t0 < tend; t0 += kRbTok) {
+#pragma unroll
+    for (int j = 0; j < XV; ++j) {
+      const int vid = tid + 64 * j;
+      const int tt = vid / (kRbTile / VE), cv = vid % (kRbTile / VE);
+#pragma unroll
+      for (int q = 0; q < VE; q += 4)
+        *reinterpret_cast<float4*>(&sx[tt][cv * VE + q]) =
+            make_float4(xr[j].get(q), xr[j].get(q + 1), xr[j].get(q + 2), xr[j].get(q + 3));
+    }
+#pragma unroll
+    for (int j = 0; j < ZV; ++j) {
+      const int vid = tid + 64 * j;
+      const int tt = vid / (kRbTile / 4), ev = vid % (kRbTile / 4);
+      *reinterpret_cast<float4*>(&sz[tt][ev * 4]) = zr[j];
     }
     __syncthreads();
+    if (t0 + kRbTok < tend) load_stage(t0 + kRbTok);
 #pragma unroll 4
     for (int tt = 0; tt < kRbTok; ++tt) {
-      const float4 zv = *reinterpret_cast<const float4*>(&sz[tt][te * 4]);
-      const float4 xv = *reinterpret_cast<const float4*>(&sx[tt][tc * 4]);
-      const float za[4] = {zv.x, zv.y, zv.z, zv.w};
-      const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float4 za = *reinterpret_cast<const float4*>(&sz[tt][te * 8]);
+      const float4 zb = *reinterpret_cast<const float4*>(&sz[tt][te * 8 + 4]);
+      const float4 xa = *reinterpret_cast<const float4*>(&sx[tt][tc * 8]);
+      const float4 xb = *reinterpret_cast<const float4*>(&sx[tt][tc * 8 + 4]);
+      const float zv[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+      for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(za[a], xa[b], acc[a][b]);
+        for (int c = 0; c < 8; ++c) acc[a][c] = __fmaf_rn(zv[a], xv[c], acc[a][c]);
     }
-    if (blockIdx.x == 0 && tid < kRbTile)
+    if (blockIdx.x == 0)
       for (int tt = 0; tt < kRbTok; ++tt) dbacc += sz[tt][tid];
     __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 4; ++a) {
-    const int e = e0 + te * 4 + a;
+  for (int a = 0; a < 8; ++a) {
+    const int e = e0 + te * 8 + a;
     if (e >= E) continue;
+    float* dst = partial + (static_cast<int64_t>(split) * E + e) * d + c0 + tc * 8;
+    if (c0 + tc * 8 + 8 <= d) {
+      reinterpret_cast<float4*>(dst)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+    } else {
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int c = c0 + tc * 4 + b;
-      if (c < d) partial[(static_cast<int64_t>(split) * E + e) * d + c] = acc[a][b];
+      for (int c = 0; c < 8; ++c)
+        if (c0 + tc * 8 + c < d) dst[c] = acc[a][c];
     }
   }
-  if (blockIdx.x == 0 && tid < kRbTile && e0 + tid < E)
-    partial_db[static_cast<int64_t>(split) * E + e0 + tid] = dbacc;
+  if (blockIdx.x == 0 && e0 + tid < E) partial_db[static_cast<int64_t>(split) * E + e0 + tid] = dbacc;
 }
 
 __global__ void router_wgrad_reduce_kernel(const float* __restrict__ partial,
@@ -395,7 +452,7 @@ __global__ void router_wgrad_reduce_kernel(const float* __restrict__ partial,
 
 int router_bwd_splits(int64_t T, int d, int E) {
   const int64_t tiles = static_cast<int64_t>((d + kRbTile - 1) / kRbTile) * ((E + kRbTile - 1) / kRbTile);
-  int64_t S = (2 * 148 + tiles - 1) / tiles;
+  int64_t S = (4 * 148 + tiles - 1) / tiles;
   const int64_t max_s = (T + kRbTok - 1) / kRbTok;
   if (S > max_s) S = max_s;
   if (S < 1) S = 1;
@@ -411,10 +468,10 @@ cudaError_t launch_router_bwd(const void* x, const float* dz, int dtype, int64_t
   float* partial_db = partial + static_cast<int64_t>(S) * E * d;
   dim3 grid((d + kRbTile - 1) / kRbTile, S, (E + kRbTile - 1) / kRbTile);
   if (dtype == MOE_BF16)
-    router_wgrad_partial_kernel<bf16><<<grid, 256, 0, s>>>(static_cast<const bf16*>(x), dz, T, d,
+    router_wgrad_partial_kernel<bf16><<<grid, 64, 0, s>>>(static_cast<const bf16*>(x), dz, T, d,
                                                            E, tps, partial, partial_db);
   else
-    router_wgrad_partial_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), dz, T,
+    router_wgrad_partial_kernel<float><<<grid, 64, 0, s>>>(static_cast<const float*>(x), dz, T,
                                                             d, E, tps, partial, partial_db);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

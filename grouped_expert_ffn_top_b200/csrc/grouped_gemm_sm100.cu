@@ -241,15 +241,33 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// Work an epilogue thread can start before its accumulator is ready: pull
-// the h1 / h2 values the SwiGLU backward will read into L2.
+// h1 / h2 values of 32 columns of this thread's row, loaded one chunk ahead
+// of their use by the SwiGLU-backward epilogue.
+struct EpiCarry {
+  uint4 h1[4], h2[4];
+};
+
+__device__ __forceinline__ void load_h_chunk(const Params& p, int64_t off, EpiCarry& c) {
+  const uint4* a = reinterpret_cast<const uint4*>(p.i0 + off);
+  const uint4* b = reinterpret_cast<const uint4*>(p.i1 + off);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    c.h1[i] = __ldg(a + i);
+    c.h2[i] = __ldg(b + i);
+  }
+}
+
+// Work an epilogue thread starts before its accumulator is ready: the first
+// chunk of h1 / h2 goes to registers, the rest of the row to L2.
 template <int KIND, int BN>
-__device__ __forceinline__ void epilogue_prefetch(const Params& p, const TileInfo& ti, int r) {
+__device__ __forceinline__ void epilogue_prefetch(const Params& p, const TileInfo& ti, int r,
+                                                  EpiCarry& carry) {
   if (KIND == kBwdDgradDown) {
     if (r < ti.rows) {
       const int64_t off = (static_cast<int64_t>(ti.row0) + r) * p.f + ti.n0;
       const int cols = min(BN, p.f - ti.n0);
-      for (int c = 0; c < cols; c += 64) {  // 64 bf16 = one 128-byte line
+      load_h_chunk(p, off, carry);
+      for (int c = 64; c < cols; c += 64) {  // 64 bf16 = one 128-byte line
         prefetch_l2(p.i0 + off + c);
         prefetch_l2(p.i1 + off + c);
       }
@@ -260,7 +278,7 @@ __device__ __forceinline__ void epilogue_prefetch(const Params& p, const TileInf
 // Epilogue of one tile for this thread's accumulator row r.
 template <int KIND, int BN>
 __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, uint32_t tacc,
-                                         int r) {
+                                         int r, EpiCarry& carry) {
   const int d = p.d, f = p.f;
   uint32_t u[16];
   float v[16];
@@ -299,30 +317,38 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
       }
     }
   } else if (KIND == kBwdDgradDown) {
+    // chunks of 32 columns; h1 / h2 of the next chunk load while this one
+    // is computed (the first chunk was loaded before the accumulator wait)
     const bool valid = r < ti.rows;
-    const int64_t row = static_cast<int64_t>(ti.row0) + r;
-    for (int c = 0; c < BN; c += 16) {
+    const int64_t base = (static_cast<int64_t>(ti.row0) + r) * f + ti.n0;
+    const int cols = min(BN, f - ti.n0);
+    for (int c = 0; c < BN; c += 32) {
+      EpiCarry next;
+      if (valid && c + 32 < cols) load_h_chunk(p, base + c + 32, next);
+      uint32_t u2[16];
       tmem_ld16(tacc + c, u);
+      tmem_ld16(tacc + c + 16, u2);
       tmem_ld_wait();
-      if (valid && ti.n0 + c < f) {
-        const int64_t off = row * f + ti.n0 + c;
-        const uint4* ph1 = reinterpret_cast<const uint4*>(p.i0 + off);
-        const uint4* ph2 = reinterpret_cast<const uint4*>(p.i1 + off);
-        float h1[16], h2[16], dh1[16], dh2[16];
-        unpack8_bf16(__ldg(ph1), h1);
-        unpack8_bf16(__ldg(ph1 + 1), h1 + 8);
-        unpack8_bf16(__ldg(ph2), h2);
-        unpack8_bf16(__ldg(ph2 + 1), h2 + 8);
+      if (valid && c < cols) {
+        float h1[32], h2[32], dh1[32], dh2[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float da = __uint_as_float(u[i]);
-          const float s = sigmoid_f(h1[i]);
-          dh1[i] = da * h2[i] * s * (1.0f + h1[i] * (1.0f - s));
-          dh2[i] = da * h1[i] * s;
+        for (int i = 0; i < 4; ++i) {
+          unpack8_bf16(carry.h1[i], h1 + 8 * i);
+          unpack8_bf16(carry.h2[i], h2 + 8 * i);
         }
-        store16_bf16(p.o0 + off, dh1);
-        store16_bf16(p.o1 + off, dh2);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float da = __uint_as_float(i < 16 ? u[i] : u2[i - 16]);
+          const float sg = sigmoid_f(h1[i]);
+          dh1[i] = da * h2[i] * sg * (1.0f + h1[i] * (1.0f - sg));
+          dh2[i] = da * h1[i] * sg;
+        }
+        store16_bf16(p.o0 + base + c, dh1);
+        store16_bf16(p.o0 + base + c + 16, dh1 + 16);
+        store16_bf16(p.o1 + base + c, dh2);
+        store16_bf16(p.o1 + base + c + 16, dh2 + 16);
       }
+      carry = next;
     }
   } else {  // kWgrad
     // Accumulator row m, column n is element (n, m) of the [N, M] row-major
@@ -561,11 +587,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      epilogue_prefetch<KIND, BN>(p, ti, r);
+      EpiCarry carry;
+      epilogue_prefetch<KIND, BN>(p, ti, r, carry);
       if (!wait_bounded(&tfull[acc], acc_phase, s_abort, kWaitLimit)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-      epilogue<KIND, BN>(p, ti, tacc, r);
+      epilogue<KIND, BN>(p, ti, tacc, r, carry);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }

@@ -12,65 +12,89 @@ namespace moe {
 // ------------------------------------------------------------ router logits
 //
 // z[t,e] = fma-chain over i = 0..d-1 of x[t,i] * Wr[e,i], then + b[e], in fp32.
-// Block tile: 128 tokens x TE experts; thread tile: 8 tokens x TE/8 experts.
-// Both operands are staged in shared memory as fp32, i-major, so one thread
-// reads 8 consecutive tokens and TE/8 consecutive experts with 128-bit loads.
+// Block tile: 64 tokens x TE experts, 64 threads; thread tile: 8 tokens x
+// TE/8 experts. Operands are staged as fp32 in shared memory, i-major, in
+// chunks of 64 i: each thread loads its token row's chunk with 16-byte vector
+// loads one chunk ahead (register double buffer) and writes it transposed.
 // The i loop is sequential for every output, which is what makes the result
 // bit-identical to the fixed-order definition.
 
-constexpr int kLogitTokens = 128;
-constexpr int kLogitChunk = 32;
+constexpr int kLogitTokens = 64;
+constexpr int kLogitChunk = 64;
 
 template <typename T, int TE>
-__global__ void __launch_bounds__(128) router_logits_kernel(const T* __restrict__ x,
-                                                            const T* __restrict__ Wr,
-                                                            const float* __restrict__ b,
-                                                            int64_t Ttok, int d, int E,
-                                                            float* __restrict__ z) {
-  constexpr int EPT = TE / 8;  // experts per thread
+__global__ void __launch_bounds__(64) router_logits_kernel(const T* __restrict__ x,
+                                                           const T* __restrict__ Wr,
+                                                           const float* __restrict__ b,
+                                                           int64_t Ttok, int d, int E,
+                                                           float* __restrict__ z) {
+  constexpr int VE = Vec16<T>::N;              // elements per 16-byte vector
+  constexpr int VPR = kLogitChunk / VE;        // vectors per row chunk
+  constexpr int WPT = TE * VPR / 64;           // Wr vectors per thread
+  constexpr int RE = TE / 8;                   // experts per thread
+  static_assert(TE * VPR % 64 == 0, "Wr staging");
   __shared__ __align__(16) float xs[kLogitChunk][kLogitTokens];
   __shared__ __align__(16) float ws[kLogitChunk][TE];
   const int tid = threadIdx.x;
-  const int tx = tid % 8;   // expert group
-  const int ty = tid / 8;   // token group (16 of them)
+  const int tx = tid % 8;  // expert group
+  const int ty = tid / 8;  // token group
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kLogitTokens;
   const int e0 = blockIdx.y * TE;
+  const int64_t my_t = t0 + tid;
 
-  float acc[8][EPT];
+  Vec16<T> xr[VPR], wr[WPT];
+  auto load_stage = [&](int i0) {
+#pragma unroll
+    for (int v = 0; v < VPR; ++v) {
+      const int i = i0 + v * VE;
+      if (my_t < Ttok && i < d) xr[v] = ld16_stream(x + my_t * d + i);
+      else xr[v].raw = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < WPT; ++j) {
+      const int vid = tid + 64 * j;
+      const int ee = vid % TE, v = vid / TE;
+      const int e = e0 + ee, i = i0 + v * VE;
+      if (e < E && i < d) wr[j] = ld16(Wr + static_cast<int64_t>(e) * d + i);
+      else wr[j].raw = make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
+
+  float acc[8][RE];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int c = 0; c < EPT; ++c) acc[a][c] = 0.0f;
+    for (int c = 0; c < RE; ++c) acc[a][c] = 0.0f;
 
+  load_stage(0);
   for (int i0 = 0; i0 < d; i0 += kLogitChunk) {
-    // stage x[t0 .. t0+127][i0 .. i0+31] transposed into xs[i][t]
-    // consecutive threads take consecutive tokens: conflict-free shared stores;
-    // the strided global reads of one row are served from L1 across ii
-    for (int idx = tid; idx < kLogitTokens * kLogitChunk; idx += 128) {
-      int tt = idx % kLogitTokens, ii = idx / kLogitTokens;
-      int64_t t = t0 + tt;
-      int i = i0 + ii;
-      xs[ii][tt] = (t < Ttok && i < d) ? to_f32(x[t * d + i]) : 0.0f;
-    }
-    for (int idx = tid; idx < TE * kLogitChunk; idx += 128) {
-      int ee = idx % TE, ii = idx / TE;
-      int e = e0 + ee, i = i0 + ii;
-      ws[ii][ee] = (e < E && i < d) ? to_f32(Wr[static_cast<int64_t>(e) * d + i]) : 0.0f;
+#pragma unroll
+    for (int v = 0; v < VPR; ++v)
+#pragma unroll
+      for (int q = 0; q < VE; ++q) xs[v * VE + q][tid] = xr[v].get(q);
+#pragma unroll
+    for (int j = 0; j < WPT; ++j) {
+      const int vid = tid + 64 * j;
+      const int ee = vid % TE, v = vid / TE;
+#pragma unroll
+      for (int q = 0; q < VE; ++q) ws[v * VE + q][ee] = wr[j].get(q);
     }
     __syncthreads();
+    if (i0 + kLogitChunk < d) load_stage(i0 + kLogitChunk);
     const int iend = min(kLogitChunk, d - i0);
+#pragma unroll 4
     for (int ii = 0; ii < iend; ++ii) {
-      float xv[8], wv[EPT];
+      float xv[8], wv[RE];
       const float4 xa = *reinterpret_cast<const float4*>(&xs[ii][ty * 8]);
       const float4 xb = *reinterpret_cast<const float4*>(&xs[ii][ty * 8 + 4]);
       xv[0] = xa.x; xv[1] = xa.y; xv[2] = xa.z; xv[3] = xa.w;
       xv[4] = xb.x; xv[5] = xb.y; xv[6] = xb.z; xv[7] = xb.w;
 #pragma unroll
-      for (int c = 0; c < EPT; ++c) wv[c] = ws[ii][tx * EPT + c];
+      for (int c = 0; c < RE; ++c) wv[c] = ws[ii][tx * RE + c];
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int c = 0; c < EPT; ++c) acc[a][c] = __fmaf_rn(xv[a], wv[c], acc[a][c]);
+        for (int c = 0; c < RE; ++c) acc[a][c] = __fmaf_rn(xv[a], wv[c], acc[a][c]);
     }
     __syncthreads();
   }
@@ -79,8 +103,8 @@ __global__ void __launch_bounds__(128) router_logits_kernel(const T* __restrict_
     const int64_t t = t0 + ty * 8 + a;
     if (t >= Ttok) continue;
 #pragma unroll
-    for (int c = 0; c < EPT; ++c) {
-      const int e = e0 + tx * EPT + c;
+    for (int c = 0; c < RE; ++c) {
+      const int e = e0 + tx * RE + c;
       if (e < E) z[t * E + e] = __fadd_rn(acc[a][c], b ? b[e] : 0.0f);
     }
   }
@@ -91,13 +115,13 @@ static cudaError_t launch_router_logits_t(const T* x, const T* Wr, const float* 
                                           int d, int E, float* z, cudaStream_t s) {
   const unsigned gx = static_cast<unsigned>((Ttok + kLogitTokens - 1) / kLogitTokens);
   if (E <= 8) {
-    router_logits_kernel<T, 8><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 8><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 16) {
-    router_logits_kernel<T, 16><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 16><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 32) {
-    router_logits_kernel<T, 32><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 32><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else {
-    router_logits_kernel<T, 64><<<dim3(gx, (E + 63) / 64), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 64><<<dim3(gx, (E + 63) / 64), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   }
   return cudaGetLastError();
 }

@@ -1,0 +1,103 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+symbol include/moe.h declares, and rejects invalid arguments with the
+documented codes before touching CUDA (no kernel is launched here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from grouped_expert_ffn_top_b200 import native as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(N.LIB_PATH):
+        from grouped_expert_ffn_top_b200 import build
+        build.build()
+    return N.lib()
+
+
+def test_header_declares_the_path():
+    syms = declared_symbols()
+    for name in ("moe_router_logits", "moe_route", "moe_permute", "moe_grouped_ffn_fwd",
+                 "moe_unpermute_combine", "moe_unpermute_combine_bwd", "moe_route_bwd",
+                 "moe_grouped_ffn_bwd", "moe_grouped_ffn_dgrad", "moe_grouped_ffn_wgrad",
+                 "moe_permute_bwd", "moe_router_bwd", "moe_get_error", "moe_last_error"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert set(declared_symbols()) <= set(N.exported_symbols()) | {"moe_launch_count"}
+
+
+def test_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {N.LIB_PATH}").read()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert exported == set(declared_symbols())
+
+
+def test_version_and_counter(L):
+    assert L.moe_version() == 1
+    assert L.moe_launch_count() >= 0
+
+
+def test_workspace_sizes(L):
+    assert L.moe_route_workspace_bytes(0, 8) >= 256
+    big = L.moe_route_workspace_bytes(32768, 64)
+    assert big >= 256 + 2 * 4 * (32768 // 256) * 64
+    assert L.moe_route_workspace_bytes(-1, 8) == 0
+    assert L.moe_grouped_ffn_bwd_workspace_bytes(1000, 8, 256, 384, N.MOE_BF16) >= 2 * 1000 * 384 * 2
+    assert L.moe_router_bwd_workspace_bytes(4096, 1024, 8) >= 256 + 4 * 8 * 1025
+
+
+null = ctypes.c_void_p(0)
+
+
+def test_route_argument_errors(L):
+    code = L.moe_route(null, 4, 8, 9, 1, *([null] * 8), null, 0, null)
+    assert code == N.MOE_ERR_INVALID_ARG
+    assert b"k=9" in L.moe_last_error()
+    assert L.moe_route(null, 4, 8, 0, 1, *([null] * 8), null, 0, null) == N.MOE_ERR_INVALID_ARG
+    assert L.moe_route(null, 4, 6, 2, 4, *([null] * 8), null, 0, null) == N.MOE_ERR_UNSUPPORTED
+    assert L.moe_route(null, 4, 2048, 2, 1, *([null] * 8), null, 0, null) == N.MOE_ERR_UNSUPPORTED
+    assert L.moe_route(null, 4, 64, 33, 1, *([null] * 8), null, 0, null) == N.MOE_ERR_UNSUPPORTED
+    # T = 0 is valid and launches nothing, even with null pointers
+    assert L.moe_route(null, 0, 8, 2, 1, *([null] * 8), null, 0, null) == N.MOE_OK
+    # null outputs with T > 0
+    assert L.moe_route(null, 4, 8, 2, 1, *([null] * 8), null, 0, null) == N.MOE_ERR_INVALID_ARG
+
+
+def test_ffn_argument_errors(L):
+    args = [null] * 4 + [N.MOE_BF16, null, 100, 4, 100, 128] + [null] * 4 + [null, 0, null]
+    assert L.moe_grouped_ffn_fwd(*args) == N.MOE_ERR_UNSUPPORTED  # d % 64 != 0 for bf16
+    args = [null] * 4 + [7, null, 100, 4, 128, 128] + [null] * 4 + [null, 0, null]
+    assert L.moe_grouped_ffn_fwd(*args) == N.MOE_ERR_UNSUPPORTED  # unknown dtype
+    args = [null] * 4 + [N.MOE_BF16, null, 0, 4, 128, 128] + [null] * 4 + [null, 0, null]
+    assert L.moe_grouped_ffn_fwd(*args) == N.MOE_OK  # no rows: nothing to do
+    args = [null] * 4 + [N.MOE_BF16, null, 10, 4, 128, 128] + [null] * 4 + [null, 0, null]
+    assert L.moe_grouped_ffn_fwd(*args) == N.MOE_ERR_INVALID_ARG  # null pointers
+    args = [null] * 4 + [N.MOE_F32, null, 10, 4, 130, 128] + [null] * 4 + [null, 0, null]
+    assert L.moe_grouped_ffn_fwd(*args) == N.MOE_ERR_UNSUPPORTED  # fp32 needs multiples of 4
+
+
+def test_row_pass_argument_errors(L):
+    assert L.moe_permute(null, N.MOE_BF16, 4, 100, 2, null, null, null) == N.MOE_ERR_UNSUPPORTED
+    assert L.moe_permute(null, N.MOE_BF16, -1, 128, 2, null, null, null) == N.MOE_ERR_INVALID_ARG
+    assert L.moe_permute(null, N.MOE_BF16, 0, 128, 2, null, null, null) == N.MOE_OK
+    assert L.moe_unpermute_combine(null, null, null, N.MOE_BF16, 4, 128, 40, null, null) == \
+        N.MOE_ERR_UNSUPPORTED
+    assert L.moe_permute_bwd(null, null, null, null, null, N.MOE_BF16, 4, 128, 2, 3, null, null) == \
+        N.MOE_ERR_INVALID_ARG  # k > E
+    assert L.moe_route_bwd(null, null, null, 4, 8, 9, null, null) == N.MOE_ERR_INVALID_ARG
+    assert L.moe_router_bwd(null, null, N.MOE_BF16, 0, 128, 8, null, null, null, 0, null) == N.MOE_OK
