@@ -17,10 +17,13 @@
 // K (the expert's rows): in the last K block the rows past the expert's end
 // are zeroed in shared memory before the MMA reads them.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM
-// and issues tcgen05.mma (one lane), warps 2-5 run the epilogue, each on its
-// TMEM lane quarter (warp % 4). Two TMEM accumulators let the epilogue of one
-// tile overlap the main loop of the next.
+// Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and issues
+// tcgen05.mma (one lane), the remaining warps run the epilogue, each on its
+// TMEM lane quarter (warp % 4). The backward kinds, whose epilogues move the
+// most memory (SwiGLU backward, fp32 weight-gradient reductions), use eight
+// epilogue warps: two per lane quarter, one per half of the tile's columns.
+// Two TMEM accumulators let the epilogue of one tile overlap the main loop
+// of the next.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -34,7 +37,11 @@ using namespace sm100;
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
-constexpr int kThreads = 192;
+template <int KIND>
+struct Roles {
+  static constexpr int kEpiWarps = (KIND == 2 || KIND == 4) ? 8 : 4;  // dgrad-down, wgrad
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+};
 constexpr int kMaxE = MOE_MAX_EXPERTS;
 constexpr long long kWaitLimit = 2000000000LL;  // about one second of SM cycles
 constexpr uint32_t kTmemCols = 512;
@@ -261,13 +268,13 @@ __device__ __forceinline__ void load_h_chunk(const Params& p, int64_t off, EpiCa
 // chunk of h1 / h2 goes to registers, the rest of the row to L2.
 template <int KIND, int BN>
 __device__ __forceinline__ void epilogue_prefetch(const Params& p, const TileInfo& ti, int r,
-                                                  EpiCarry& carry) {
+                                                  int c0, EpiCarry& carry) {
   if (KIND == kBwdDgradDown) {
-    if (r < ti.rows) {
+    const int cols = min(c0 + BN / 2, p.f - ti.n0);
+    if (r < ti.rows && c0 < cols) {
       const int64_t off = (static_cast<int64_t>(ti.row0) + r) * p.f + ti.n0;
-      const int cols = min(BN, p.f - ti.n0);
-      load_h_chunk(p, off, carry);
-      for (int c = 64; c < cols; c += 64) {  // 64 bf16 = one 128-byte line
+      load_h_chunk(p, off + c0, carry);
+      for (int c = c0 + 64; c < cols; c += 64) {  // 64 bf16 = one 128-byte line
         prefetch_l2(p.i0 + off + c);
         prefetch_l2(p.i1 + off + c);
       }
@@ -275,17 +282,20 @@ __device__ __forceinline__ void epilogue_prefetch(const Params& p, const TileInf
   }
 }
 
-// Epilogue of one tile for this thread's accumulator row r.
+// Epilogue of one tile for this thread's accumulator row r, on the columns
+// [c0, c0 + W) of the accumulator, W = BN / (epilogue warps / 4) (the gate/up
+// kind: f columns [c0, c0 + 128 / split), each with its gate and up
+// accumulator).
 template <int KIND, int BN>
 __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, uint32_t tacc,
-                                         int r, EpiCarry& carry) {
+                                         int r, int c0, EpiCarry& carry) {
   const int d = p.d, f = p.f;
   uint32_t u[16];
   float v[16];
   if (KIND == kFwdGateUp) {
     const bool valid = r < ti.rows;
     const int64_t row = static_cast<int64_t>(ti.row0) + r;
-    for (int c = 0; c < 128; c += 16) {
+    for (int c = c0; c < c0 + 128 / (Roles<KIND>::kEpiWarps / 4); c += 16) {
       uint32_t g[16];
       tmem_ld16(tacc + c, g);
       tmem_ld16(tacc + 128 + c, u);
@@ -307,7 +317,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
   } else if (KIND == kFwdDown || KIND == kBwdDgradGateUp) {
     const bool valid = r < ti.rows;
     const int64_t row = static_cast<int64_t>(ti.row0) + r;
-    for (int c = 0; c < BN; c += 16) {
+    for (int c = c0; c < c0 + BN / (Roles<KIND>::kEpiWarps / 4); c += 16) {
       tmem_ld16(tacc + c, u);
       tmem_ld_wait();
       if (valid && ti.n0 + c < d) {
@@ -321,8 +331,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
     // is computed (the first chunk was loaded before the accumulator wait)
     const bool valid = r < ti.rows;
     const int64_t base = (static_cast<int64_t>(ti.row0) + r) * f + ti.n0;
-    const int cols = min(BN, f - ti.n0);
-    for (int c = 0; c < BN; c += 32) {
+    const int cols = min(c0 + BN / 2, f - ti.n0);
+    for (int c = c0; c < c0 + BN / 2; c += 32) {
       EpiCarry next;
       if (valid && c + 32 < cols) load_h_chunk(p, base + c + 32, next);
       uint32_t u2[16];
@@ -362,7 +372,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
     const bool valid = m < M;
     float* out = (ti.prod == 0 ? p.w0 : (ti.prod == 1 ? p.w1 : p.w2)) +
                  static_cast<int64_t>(ti.e) * d * f + m;
-    for (int c = 0; c < BN; c += 16) {
+    for (int c = c0; c < c0 + BN / 2; c += 16) {
       tmem_ld16(tacc + c, u);
       tmem_ld_wait();
       if (valid && ti.n0 + c < Nn) {
@@ -375,7 +385,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
 }
 
 template <int KIND, int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
   using Tr = Traits<KIND, BN>;
   constexpr int STAGES = Tr::STAGES;
@@ -389,8 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + 2;
-  uint64_t* aux = tempty + 2;
-  uint64_t* drain = aux + 1;
+  uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort) + 1;
@@ -410,9 +419,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 32 * Roles<KIND>::kEpiWarps);
     }
-    mbar_init(aux, 1);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -429,10 +437,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(s_tmem, kTmemCols);
     tmem_relinquish();
   }
-  for (int e = threadIdx.x; e <= E; e += kThreads) s_off[e] = p.offsets[e];
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = p.offsets[e];
   __syncthreads();
   // schedule order: wgrad tiles have ragged K, so experts go longest first
-  for (int e = threadIdx.x; e < E; e += kThreads) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
     if (KIND == kWgrad) {
       const int64_t c = s_off[e + 1] - s_off[e];
       int rank = 0;
@@ -479,9 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     int stage = 0;
-    uint32_t phase = 0, aux_phase = 0;
+    uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // last load issued on full[s], and its phase
-    bool aux_pending = false;
     for (int tile = blockIdx.x; tile < total && !*s_abort; tile += gridDim.x) {
       const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
@@ -489,34 +496,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, kWaitLimit)) break;
         uint8_t* a_dst = sA + stage * Tr::A_BYTES;
         uint8_t* b_dst = sB + stage * Tr::B_BYTES;
-        const bool tail = (KIND == kWgrad) && ((kb + 1) * BK > ti.rows);
-        uint64_t* bar = tail ? aux : &full[stage];
         if (lane == 0) {
-          mbar_arrive_expect_tx(bar, Tr::STAGE_TX);
-          issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, bar);
+          mbar_arrive_expect_tx(&full[stage], Tr::STAGE_TX);
+          issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
         }
-        if (!tail) {
-          issued_mask |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-        }
-        if (tail) {
-          // rows past the expert's end belong to the next expert (or lie past
-          // the tensor): zero them in both operands so they add nothing
-          aux_pending = true;
-          if (!wait_bounded(aux, aux_phase, s_abort, kWaitLimit)) break;
-          aux_pending = false;
-          aux_phase ^= 1u;
-          const int valid = ti.rows - kb * BK;
-          const int chunks = (BK - valid) * 8;  // 16-byte chunks per 8 KB box
-          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          for (int box = 0; box < 2 + BN / 64; ++box) {
-            uint8_t* base = (box < 2 ? a_dst + box * 8192 : b_dst + (box - 2) * 8192) + valid * 128;
-            for (int c = lane; c < chunks; c += 32) reinterpret_cast<uint4*>(base)[c] = z;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&full[stage]);
-        }
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -528,7 +513,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       volatile int never = 0;
       for (int s = 0; s < STAGES; ++s)
         if ((issued_mask >> s) & 1u) wait_bounded(&full[s], (issued_par >> s) & 1u, &never, kWaitLimit);
-      if (aux_pending) wait_bounded(aux, aux_phase, &never, kWaitLimit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
@@ -550,11 +534,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        int ksteps = BK / 16;
+        if (KIND == kWgrad && (kb + 1) * BK > ti.rows) {
+          // ragged-K tail: rows past the expert's end belong to the next
+          // expert (or lie past the tensor). Only the 16-row MMA steps that
+          // hold valid rows run, and the invalid rows inside the last of them
+          // are zeroed in both operands first.
+          const int valid = ti.rows - kb * BK;
+          ksteps = (valid + 15) / 16;
+          const int zrows = ksteps * 16 - valid;
+          if (zrows > 0) {
+            uint8_t* a_st = sA + stage * Tr::A_BYTES;
+            uint8_t* b_st = sB + stage * Tr::B_BYTES;
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            const int chunks = zrows * 8;  // 16-byte chunks per 64-column box
+            for (int box = 0; box < 2 + BN / 64; ++box) {
+              uint8_t* base = (box < 2 ? a_st + box * 8192 : b_st + (box - 2) * 8192) + valid * 128;
+              for (int c = lane; c < chunks; c += 32) reinterpret_cast<uint4*>(base)[c] = z;
+            }
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+        }
         if (lane == 0) {
           const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
+            if (kk >= ksteps) break;
             const uint64_t adesc = Tr::A_MN ? umma_desc_sw128(a_addr + kk * 2048, 8192, 1024)
                                             : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bdesc = Tr::B_MN ? umma_desc_sw128(b_addr + kk * 2048, 8192, 1024)
@@ -582,17 +589,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    // with eight epilogue warps each handles half of the columns
+    constexpr int kSplit = Roles<KIND>::kEpiWarps / 4;
+    const int c0 = ((warp - 2) >> 2) * ((KIND == kFwdGateUp ? 128 : BN) / kSplit);
     int it = 0;
     for (int tile = blockIdx.x; tile < total && !*s_abort; tile += gridDim.x, ++it) {
       const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       EpiCarry carry;
-      epilogue_prefetch<KIND, BN>(p, ti, r, carry);
+      epilogue_prefetch<KIND, BN>(p, ti, r, c0, carry);
       if (!wait_bounded(&tfull[acc], acc_phase, s_abort, kWaitLimit)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-      epilogue<KIND, BN>(p, ti, tacc, r, carry);
+      epilogue<KIND, BN>(p, ti, tacc, r, c0, carry);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
     }
@@ -657,7 +667,7 @@ static cudaError_t launch(const Maps& m, const Params& p, cudaStream_t s) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Tr::SMEM));
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<KIND, BN><<<sm_count(), kThreads, Tr::SMEM, s>>>(m, p);
+  grouped_gemm_kernel<KIND, BN><<<sm_count(), Roles<KIND>::kThreads, Tr::SMEM, s>>>(m, p);
   return cudaGetLastError();
 }
 

@@ -77,6 +77,10 @@ WORKLOADS: Dict[str, Workload] = {
         "fine_fwdbwd_32k", [32768], d=2048, E=64, k=8, f=1408, dtype=BF16, bias="zipf",
         backward=True, ep_groups=4,
         description="fine-grained bf16 forward+backward on one packed 32k sequence, Zipf-skewed"),
+    "fine_fwdbwd_8k": Workload(
+        "fine_fwdbwd_8k", [8192], d=2048, E=64, k=8, f=1408, dtype=BF16, bias="zipf",
+        backward=True, ep_groups=4,
+        description="the 32k workload's layer on 8192 tokens (kernel profiling: a few GB on the device)"),
     "uneven_sweep": Workload(
         "uneven_sweep", [32768, 9000, 1, 0], d=4096, E=16, k=2, f=14336, dtype=BF16,
         bias=("normal", 1.0), backward=True, ep_groups=1,
