@@ -20,7 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 
-SOURCES = ["api.cu", "route.cu", "dispatch.cu", "grouped_gemm_sm100.cu", "grouped_simt.cu"]
+SOURCES = ["api.cu", "route.cu", "route_noalloc.cu", "dispatch.cu", "grouped_gemm_sm100.cu",
+           "grouped_simt.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -71,6 +71,14 @@ int check_ffn(const char* fn, int dtype, int64_t rows, int E, int d, int f) {
 
 }  // namespace
 
+namespace moe {
+// Records the message moe_last_error() returns, for entry points defined in
+// other files of the library; returns `code`.
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+// Adds `n` kernel launches to the count moe_launch_count() returns.
+void count_launches(int n) { counted(n); }
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_last_error(void) { return g_msg; }

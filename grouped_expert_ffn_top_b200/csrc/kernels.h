@@ -11,6 +11,10 @@ namespace moe {
 constexpr int kRouteThreads = 256;
 constexpr int kRouteTokensPerBlock = 256;
 
+// error message and launch count of the C ABI (api.cu)
+int report_error(int code, const char* msg);
+void count_launches(int n);
+
 // routing (route.cu)
 cudaError_t launch_router_logits(const void* x, const void* Wr, const float* b, int dtype,
                                  int64_t T, int d, int E, float* z, cudaStream_t s);

@@ -51,6 +51,7 @@ _SIGNATURES = {
     "moe_router_logits": ([_p, _p, _p, _i, _i64, _i, _i, _p, _p], _i),
     "moe_route_workspace_bytes": ([_i64, _i], _sz),
     "moe_route": ([_p, _i64, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_route_noalloc": ([_p, _i64, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p], _i),
     "moe_permute": ([_p, _i, _i64, _i, _i, _p, _p, _p], _i),
     "moe_grouped_ffn_fwd_workspace_bytes": ([_i64, _i, _i, _i, _i], _sz),
     "moe_grouped_ffn_fwd": ([_p, _p, _p, _p, _i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p], _i),

@@ -150,6 +150,34 @@ MOE_API int moe_route(const float* logits, int64_t T, int E, int k, int ep_group
               int32_t* row_of_pair, int32_t* pair_of_row,
               void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Largest ceil(T/256) * E that moe_route_noalloc accepts. */
+#define MOE_ROUTE_NOALLOC_MAX_SLOTS 262144
+
+/* moe_route for callers that cannot allocate device memory. (The pages have
+ * no counterpart of this entry point; it exists for integration.)
+ * moe_route asks the caller for a workspace; some callers cannot provide one:
+ * code running inside another library or runtime that owns all device memory,
+ * hosts that plan every byte ahead and forbid new allocations, or paths where
+ * a cudaMalloc would synchronise the device. This variant keeps its scratch
+ * (per-block expert counts and bases) in a fixed array compiled into the
+ * library -- 2 MiB per GPU that loads the library, held until the process
+ * exits -- and calls no cudaMalloc, cudaFree or other allocating routine.
+ * Same arguments, outputs and results as moe_route, except:
+ *   - no workspace; ceil(T/256) * E must not exceed MOE_ROUTE_NOALLOC_MAX_SLOTS
+ *     (MOE_ERR_UNSUPPORTED otherwise: use moe_route);
+ *   - err_flags: device pointer to a caller-zeroed unsigned int that the
+ *     kernels OR MOE_DEVERR_* bits into, or NULL to not report them.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make it before any stream capture. All calls on a
+ * device share the array: calls that overlap on the GPU (other streams,
+ * other host threads) race, so the caller must serialise them. Nothing has
+ * to be cleared between calls. */
+MOE_API int moe_route_noalloc(const float* logits, int64_t T, int E, int k, int ep_groups,
+                              int32_t* topk_idx, float* topk_w, int32_t* expert_counts,
+                              int64_t* expert_offsets, int32_t* group_counts,
+                              int64_t* group_offsets, int32_t* row_of_pair, int32_t* pair_of_row,
+                              unsigned int* err_flags, cudaStream_t stream);
+
 /* ---------------------------------------------------------- dispatch */
 
 /* Permute (dispatch copy): xp[row_of_pair[t*k+j], :] = x[t, :].
