@@ -87,6 +87,15 @@ int moe_version(void) { return 1; }
 
 int64_t moe_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int moe_selftest_wait_timeout(void* ws, long long limit_cycles, cudaStream_t stream) {
+  if (!ws || !aligned16(ws)) return fail(MOE_ERR_INVALID_ARG, "moe_selftest_wait_timeout: workspace");
+  if (limit_cycles < 1000) limit_cycles = 1000;
+  if (limit_cycles > 4000000000LL) limit_cycles = 4000000000LL;
+  return launched(cuda_status(moe::launch_selftest_wait_timeout(static_cast<unsigned*>(ws),
+                                                                limit_cycles, stream),
+                              "moe_selftest_wait_timeout"), 1);
+}
+
 int moe_get_error(void* ws, cudaStream_t stream) {
   if (!ws) return fail(MOE_ERR_INVALID_ARG, "moe_get_error: null workspace");
   unsigned h = 0;
@@ -222,24 +231,29 @@ int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dl
                      "moe_permute_bwd") == MOE_OK ? launched(MOE_OK, 1) : MOE_ERR_CUDA;
 }
 
-size_t moe_router_bwd_workspace_bytes(int64_t T, int d, int E) {
-  if (T < 0 || d < 1 || E < 1) return 0;
-  const int S = moe::router_bwd_splits(T, d, E);
-  return moe::kWsHeader + align256(sizeof(float) * static_cast<size_t>(S) * E * (d + 1));
+size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E) {
+  if (rows < 0 || d < 1 || E < 1) return 0;
+  const size_t items = static_cast<size_t>(moe::router_bwd_max_items(rows, E));
+  return moe::kWsHeader + align256(sizeof(float) * items * (static_cast<size_t>(d) + 1));
 }
 
-int moe_router_bwd(const void* x, const float* dlogits, int dtype, int64_t T, int d, int E,
+int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_row,
+                   const int64_t* expert_offsets, int dtype, int64_t T, int d, int E, int k,
                    float* dWr, float* db, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  if (!dtype_ok(dtype)) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd: dtype %d", dtype);
-  if (T < 0 || d < 1 || E < 1) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: sizes");
+  int rc = check_rows("moe_router_bwd", dtype, T, d, k);
+  if (rc != MOE_OK) return rc;
+  if (E < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: E=%d k=%d", E, k);
   if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd: E=%d", E);
   if (T == 0) return MOE_OK;
-  if (!x || !dlogits || !dWr || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: null pointer");
-  if (ws_bytes < moe_router_bwd_workspace_bytes(T, d, E) || !aligned16(ws))
-    return fail(MOE_ERR_WORKSPACE, "moe_router_bwd: workspace needs %zu bytes",
-                moe_router_bwd_workspace_bytes(T, d, E));
+  if (!xp || !dlogits || !pair_of_row || !expert_offsets || !dWr || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: null pointer");
+  const int64_t rows = T * k;
+  if (ws_bytes < moe_router_bwd_workspace_bytes(rows, d, E) || !aligned16(ws) || !aligned16(xp))
+    return fail(MOE_ERR_WORKSPACE, "moe_router_bwd: workspace needs %zu bytes (16-byte aligned)",
+                moe_router_bwd_workspace_bytes(rows, d, E));
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + moe::kWsHeader);
-  return launched(cuda_status(moe::launch_router_bwd(x, dlogits, dtype, T, d, E, dWr, db, partial,
+  return launched(cuda_status(moe::launch_router_bwd(xp, dlogits, pair_of_row, expert_offsets,
+                                                      dtype, rows, d, E, k, dWr, db, partial,
                                                       stream),
                               "moe_router_bwd"), 2);
 }

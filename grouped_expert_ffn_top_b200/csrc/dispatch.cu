@@ -316,168 +316,132 @@ cudaError_t launch_permute_bwd(const void* dxp, const int32_t* row_of_pair, cons
 // split into partial[split][e][c] (fp32). Pass 2 adds the splits in order.
 // No atomics: the result does not depend on scheduling.
 
-constexpr int kRbTile = 64;
-constexpr int kRbTok = 32;
+constexpr int kRbRows = 256;  // dispatch rows per work item
+constexpr int kRbThreads = 256;
 
-// Block: 64 experts x 64 columns of dWr, 64 threads, 8x8 register tile per
-// thread; tokens of the block's split in chunks of 32, staged with 16-byte
-// loads one chunk ahead (register double buffer).
-template <typename T>
-__global__ void __launch_bounds__(64) router_wgrad_partial_kernel(
-    const T* __restrict__ x, const float* __restrict__ dz, int64_t Ttok, int d, int E,
-    int64_t tok_per_split, float* __restrict__ partial, float* __restrict__ partial_db) {
-  constexpr int VE = Vec16<T>::N;
-  constexpr int XV = kRbTok * kRbTile / VE / 64;  // x vectors per thread per chunk
-  constexpr int ZV = kRbTok * kRbTile / 4 / 64;   // dz float4 per thread per chunk
-  __shared__ __align__(16) float sz[kRbTok][kRbTile];
-  __shared__ __align__(16) float sx[kRbTok][kRbTile];
-  const int tid = threadIdx.x;
-  const int te = tid / 8, tc = tid % 8;
-  const int c0 = blockIdx.x * kRbTile;
-  const int split = blockIdx.y;
-  const int e0 = blockIdx.z * kRbTile;
-  const int64_t tb = split * tok_per_split;
-  const int64_t tend = min(Ttok, tb + tok_per_split);
-  const bool e_vec_ok = (E % 4 == 0);
-
-  Vec16<T> xr[XV];
-  float4 zr[ZV];
-  auto load_stage = [&](int64_t t0) {
-#pragma unroll
-    for (int j = 0; j < XV; ++j) {
-      const int vid = tid + 64 * j;
-      const int tt = vid / (kRbTile / VE), cv = vid % (kRbTile / VE);
-      const int64_t t = t0 + tt;
-      const int c = c0 + cv * VE;
-      if (t < tend && c < d) xr[j] = ld16_stream(x + t * d + c);
-      else xr[j].raw = make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int j = 0; j < ZV; ++j) {
-      const int vid = tid + 64 * j;
-      const int tt = vid / (kRbTile / 4), ev = vid % (kRbTile / 4);
-      const int64_t t = t0 + tt;
-      const int e = e0 + ev * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t < tend) {
-        const float* src = dz + t * E + e;
-        if (e_vec_ok && e + 3 < E) {
-          v = __ldcs(reinterpret_cast<const float4*>(src));
-        } else {
-          if (e < E) v.x = src[0];
-          if (e + 1 < E) v.y = src[1];
-          if (e + 2 < E) v.z = src[2];
-          if (e + 3 < E) v.w = src[3];
-        }
-      }
-      zr[j] = v;
-    }
-  };
-
-  float acc[8][8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) acc[a][c] = 0.0f;
-  float dbacc = 0.0f;
-  if (tb < tend) load_stage(tb);
-  for (int64_t t0 = tb; t0 < tend; t0 += kRbTok) {
-#pragma unroll
-    for (int j = 0; j < XV; ++j) {
-      const int vid = tid + 64 * j;
-      const int tt = vid / (kRbTile / VE), cv = vid % (kRbTile / VE);
-#pragma unroll
-      for (int q = 0; q < VE; q += 4)
-        *reinterpret_cast<float4*>(&sx[tt][cv * VE + q]) =
-            make_float4(xr[j].get(q), xr[j].get(q + 1), xr[j].get(q + 2), xr[j].get(q + 3));
-    }
-#pragma unroll
-    for (int j = 0; j < ZV; ++j) {
-      const int vid = tid + 64 * j;
-      const int tt = vid / (kRbTile / 4), ev = vid % (kRbTile / 4);
-      *reinterpret_cast<float4*>(&sz[tt][ev * 4]) = zr[j];
-    }
-    __syncthreads();
-    if (t0 + kRbTok < tend) load_stage(t0 + kRbTok);
-#pragma unroll 4
-    for (int tt = 0; tt < kRbTok; ++tt) {
-      const float4 za = *reinterpret_cast<const float4*>(&sz[tt][te * 8]);
-      const float4 zb = *reinterpret_cast<const float4*>(&sz[tt][te * 8 + 4]);
-      const float4 xa = *reinterpret_cast<const float4*>(&sx[tt][tc * 8]);
-      const float4 xb = *reinterpret_cast<const float4*>(&sx[tt][tc * 8 + 4]);
-      const float zv[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[a][c] = __fmaf_rn(zv[a], xv[c], acc[a][c]);
-    }
-    if (blockIdx.x == 0)
-      for (int tt = 0; tt < kRbTok; ++tt) dbacc += sz[tt][tid];
-    __syncthreads();
-  }
-#pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int e = e0 + te * 8 + a;
-    if (e >= E) continue;
-    float* dst = partial + (static_cast<int64_t>(split) * E + e) * d + c0 + tc * 8;
-    if (c0 + tc * 8 + 8 <= d) {
-      reinterpret_cast<float4*>(dst)[0] = make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-      reinterpret_cast<float4*>(dst)[1] = make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
-    } else {
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        if (c0 + tc * 8 + c < d) dst[c] = acc[a][c];
-    }
-  }
-  if (blockIdx.x == 0 && e0 + tid < E) partial_db[static_cast<int64_t>(split) * E + e0 + tid] = dbacc;
+int router_bwd_max_items(int64_t rows, int E) {
+  return static_cast<int>((rows + kRbRows - 1) / kRbRows) + E;
 }
 
-__global__ void router_wgrad_reduce_kernel(const float* __restrict__ partial,
-                                           const float* __restrict__ partial_db, int S, int E,
-                                           int d, float* __restrict__ dWr, float* __restrict__ db) {
+// First work item of each expert (expert e owns ceil(count_e / kRbRows)
+// items, in expert order); s_start[E] = number of items. Whole block.
+__device__ void router_items_prefix(const int64_t* __restrict__ off, int E, int* s_start) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    int carry = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int v = e < E ? static_cast<int>((off[e + 1] - off[e] + kRbRows - 1) / kRbRows) : 0;
+      int inc = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
+      }
+      if (e < E) s_start[e] = carry + inc - v;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) s_start[E] = carry;
+  }
+  __syncthreads();
+}
+
+__device__ __forceinline__ int expert_of_item(const int* s_start, int E, int item) {
+  int lo = 0, hi = E - 1;  // largest e with s_start[e] <= item
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_start[mid] <= item) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// partial[item, cols] = sum over the item's rows r (ascending) of
+// dz[token(r), e] * xp[r, cols]; partial_db[item] = sum of those dz.
+// Each xp row is read once, 16 bytes per thread, coalesced across the block.
+template <typename T>
+__global__ void __launch_bounds__(kRbThreads) router_wgrad_partial_kernel(
+    const T* __restrict__ xp, const float* __restrict__ dz, const int32_t* __restrict__ por,
+    const int64_t* __restrict__ off, int E, int d, int k, float* __restrict__ partial,
+    float* __restrict__ partial_db) {
+  constexpr int VE = Vec16<T>::N;
+  __shared__ int s_start[MOE_MAX_EXPERTS + 1];
+  __shared__ float s_dz[kRbRows];
+  router_items_prefix(off, E, s_start);
+  const int item = blockIdx.x;
+  if (item >= s_start[E]) return;
+  const int e = expert_of_item(s_start, E, item);
+  const int64_t r0 = off[e] + static_cast<int64_t>(item - s_start[e]) * kRbRows;
+  const int nrows = static_cast<int>(min(off[e + 1] - r0, static_cast<int64_t>(kRbRows)));
+  for (int i = threadIdx.x; i < nrows; i += blockDim.x)
+    s_dz[i] = dz[static_cast<int64_t>(por[r0 + i] / k) * E + e];
+  __syncthreads();
+  const int c = (blockIdx.y * kRbThreads + threadIdx.x) * VE;
+  if (c < d) {
+    float acc[VE];
+#pragma unroll
+    for (int q = 0; q < VE; ++q) acc[q] = 0.0f;
+    const T* src = xp + r0 * d + c;
+#pragma unroll 4
+    for (int i = 0; i < nrows; ++i) {
+      const Vec16<T> v = ld16_stream(src + static_cast<int64_t>(i) * d);
+      const float g = s_dz[i];
+#pragma unroll
+      for (int q = 0; q < VE; ++q) acc[q] = __fmaf_rn(g, v.get(q), acc[q]);
+    }
+    float* dst = partial + static_cast<int64_t>(item) * d + c;
+#pragma unroll
+    for (int q = 0; q < VE; q += 4)
+      *reinterpret_cast<float4*>(dst + q) = make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+  }
+  if (blockIdx.y == 0 && threadIdx.x == 0) {
+    float sdb = 0.0f;
+    for (int i = 0; i < nrows; ++i) sdb += s_dz[i];
+    partial_db[item] = sdb;
+  }
+}
+
+// dWr[e, c] += sum of expert e's item partials, in item order; db likewise.
+__global__ void __launch_bounds__(256) router_wgrad_reduce_kernel(
+    const float* __restrict__ partial, const float* __restrict__ partial_db,
+    const int64_t* __restrict__ off, int E, int d, float* __restrict__ dWr, float* __restrict__ db) {
+  __shared__ int s_start[MOE_MAX_EXPERTS + 1];
+  router_items_prefix(off, E, s_start);
   const int64_t n = static_cast<int64_t>(E) * d;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int e = static_cast<int>(i / d);
+    const int c = static_cast<int>(i % d);
+    if (s_start[e + 1] == s_start[e]) continue;  // no token selected e: untouched
     float s = 0.0f;
-    for (int q = 0; q < S; ++q) s += partial[q * n + i];
+    for (int it = s_start[e]; it < s_start[e + 1]; ++it) s += partial[static_cast<int64_t>(it) * d + c];
     dWr[i] += s;
-    if (db && i < E) {
+    if (db && c == 0) {
       float sb = 0.0f;
-      for (int q = 0; q < S; ++q) sb += partial_db[static_cast<int64_t>(q) * E + i];
-      db[i] += sb;
+      for (int it = s_start[e]; it < s_start[e + 1]; ++it) sb += partial_db[it];
+      db[e] += sb;
     }
   }
 }
 
-int router_bwd_splits(int64_t T, int d, int E) {
-  const int64_t tiles = static_cast<int64_t>((d + kRbTile - 1) / kRbTile) * ((E + kRbTile - 1) / kRbTile);
-  int64_t S = (4 * 148 + tiles - 1) / tiles;
-  const int64_t max_s = (T + kRbTok - 1) / kRbTok;
-  if (S > max_s) S = max_s;
-  if (S < 1) S = 1;
-  if (S > 1024) S = 1024;
-  return static_cast<int>(S);
-}
-
-cudaError_t launch_router_bwd(const void* x, const float* dz, int dtype, int64_t T, int d, int E,
+cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* por,
+                              const int64_t* off, int dtype, int64_t rows, int d, int E, int k,
                               float* dWr, float* db, float* partial, cudaStream_t s) {
-  const int S = router_bwd_splits(T, d, E);
-  int64_t tps = (T + S - 1) / S;
-  tps = (tps + kRbTok - 1) / kRbTok * kRbTok;
-  float* partial_db = partial + static_cast<int64_t>(S) * E * d;
-  dim3 grid((d + kRbTile - 1) / kRbTile, S, (E + kRbTile - 1) / kRbTile);
+  const int items = router_bwd_max_items(rows, E);
+  float* partial_db = partial + static_cast<int64_t>(items) * d;
+  const int vec = dtype == MOE_BF16 ? 8 : 4;
+  dim3 grid(items, (d + kRbThreads * vec - 1) / (kRbThreads * vec));
   if (dtype == MOE_BF16)
-    router_wgrad_partial_kernel<bf16><<<grid, 64, 0, s>>>(static_cast<const bf16*>(x), dz, T, d,
-                                                           E, tps, partial, partial_db);
+    router_wgrad_partial_kernel<bf16><<<grid, kRbThreads, 0, s>>>(
+        static_cast<const bf16*>(xp), dz, por, off, E, d, k, partial, partial_db);
   else
-    router_wgrad_partial_kernel<float><<<grid, 64, 0, s>>>(static_cast<const float*>(x), dz, T,
-                                                            d, E, tps, partial, partial_db);
+    router_wgrad_partial_kernel<float><<<grid, kRbThreads, 0, s>>>(
+        static_cast<const float*>(xp), dz, por, off, E, d, k, partial, partial_db);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(E) * d;
   const unsigned blocks = static_cast<unsigned>(((n + 255) / 256) < 148 * 8 ? (n + 255) / 256 : 148 * 8);
-  router_wgrad_reduce_kernel<<<blocks, 256, 0, s>>>(partial, partial_db, S, E, d, dWr, db);
+  router_wgrad_reduce_kernel<<<blocks, 256, 0, s>>>(partial, partial_db, off, E, d, dWr, db);
   return cudaGetLastError();
 }
 

@@ -72,15 +72,21 @@ struct Params {
   unsigned* err;
 };
 
-template <int KIND, int BN>
+// PAIR: a cluster of two CTAs computes a 256-row tile with one
+// tcgen05.mma.cta_group::2 per K step; each CTA stages its 128 rows of A and
+// half of B, so per-SM operand traffic per flop drops by a third and six
+// pipeline stages fit in shared memory.
+template <int KIND, int BN, bool PAIR = false>
 struct Traits {
   static constexpr bool A_MN = KIND == kWgrad;
   static constexpr bool B_MN = KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || KIND == kWgrad;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
-  static constexpr uint32_t A_BYTES = BM * BK * 2;
-  static constexpr uint32_t B_BYTES = BN * BK * 2;
-  static constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES;
-  static constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, A_MN, B_MN);
+  static constexpr int TM = PAIR ? 2 * BM : BM;  // rows of one tile
+  static constexpr int STAGES = (PAIR || BN != 256) ? 6 : 4;
+  static constexpr uint32_t A_BYTES = BM * BK * 2;                      // per CTA
+  static constexpr uint32_t B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;    // per CTA
+  static constexpr uint32_t STAGE_TX = (A_BYTES + B_BYTES) * (PAIR ? 2 : 1);  // all CTAs
+  static constexpr uint32_t IDESC = umma_idesc_bf16(TM, BN, A_MN, B_MN);
+  static_assert(!PAIR || KIND != kWgrad, "the ragged-K kind runs on single CTAs");
   // N extent of one output tile (gate/up: 128 f columns, each with its gate
   // and up accumulator, together the MMA's N = 256)
   static constexpr int NTILE = KIND == kFwdGateUp ? 128 : BN;
@@ -104,13 +110,13 @@ struct TileInfo {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 __device__ __forceinline__ int tiles_of_expert(int cnt, int d, int f) {
-  using Tr = Traits<KIND, BN>;
+  using Tr = Traits<KIND, BN, PAIR>;
   if (cnt <= 0) return 0;
   if (KIND == kWgrad) return 2 * ceil_div(d, BM) * ceil_div(f, BN) + ceil_div(f, BM) * ceil_div(d, BN);
   const int n_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? f : d;
-  return ceil_div(cnt, BM) * ceil_div(n_extent, Tr::NTILE);
+  return ceil_div(cnt, Tr::TM) * ceil_div(n_extent, Tr::NTILE);
 }
 
 template <int KIND, int BN>
@@ -128,9 +134,9 @@ struct Sched {
   int E;
 };
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d, int f) {
-  using Tr = Traits<KIND, BN>;
+  using Tr = Traits<KIND, BN, PAIR>;
   int lo = 0, hi = s.E - 1;
   while (lo < hi) {  // largest slot whose first tile is <= tile
     const int mid = (lo + hi + 1) >> 1;
@@ -165,8 +171,8 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d,
     const int nt = ceil_div(n_extent, Tr::NTILE);
     const int mi = local / nt;
     ti.n0 = (local % nt) * Tr::NTILE;
-    ti.row0 = base + mi * BM;
-    ti.rows = min(BM, cnt - mi * BM);
+    ti.row0 = base + mi * Tr::TM;
+    ti.rows = min(Tr::TM, cnt - mi * Tr::TM);
     ti.m0 = 0;
     ti.prod = 0;
   }
@@ -208,6 +214,39 @@ __device__ __forceinline__ void issue_loads(const Maps& m, const TileInfo& ti, i
     tma_load_2d(a_dst + 8192, am, bar, ti.m0 + 64, r);
 #pragma unroll
     for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, bm, bar, ti.n0 + 64 * j, r);
+  }
+}
+
+// The same k block for one CTA of a pair: this CTA's 128 rows of A and its
+// half of B (gate/up: CTA 0 stages the Wg rows, CTA 1 the Wu rows), counted
+// on the even CTA's mbarrier at `bar`, a shared::cluster address.
+template <int KIND, int BN>
+__device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& ti, int kb, int d,
+                                                 int f, int cta, uint8_t* a_dst, uint8_t* b_dst,
+                                                 uint32_t bar) {
+  const int k0 = kb * BK;
+  const int arow = ti.row0 + BM * cta;
+  constexpr int HALF = BN / 2;
+  if (KIND == kFwdGateUp) {
+    tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
+    tma_load_2d_pair(b_dst, cta == 0 ? &m.b0 : &m.b1, bar, k0, ti.e * f + ti.n0);
+  } else if (KIND == kFwdDown) {
+    tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
+    tma_load_2d_pair(b_dst, &m.b0, bar, k0, ti.e * d + ti.n0 + HALF * cta);
+  } else if (KIND == kBwdDgradDown) {
+    tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
+#pragma unroll
+    for (int j = 0; j < HALF / 64; ++j)
+      tma_load_2d_pair(b_dst + j * 8192, &m.b0, bar, ti.n0 + HALF * cta + 64 * j, ti.e * d + k0);
+  } else if (KIND == kBwdDgradGateUp) {
+    const int half = f / BK;
+    const bool second = kb >= half;
+    const int kk = (second ? kb - half : kb) * BK;
+    tma_load_2d_pair(a_dst, second ? &m.a1 : &m.a0, bar, kk, arow);
+#pragma unroll
+    for (int j = 0; j < HALF / 64; ++j)
+      tma_load_2d_pair(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + HALF * cta + 64 * j,
+                       ti.e * f + kk);
   }
 }
 
@@ -384,10 +423,10 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
   }
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
-  using Tr = Traits<KIND, BN>;
+  using Tr = Traits<KIND, BN, PAIR>;
   constexpr int STAGES = Tr::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -410,6 +449,11 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int E = p.E, d = p.d, f = p.f;
+  // a pair shares its tiles: tile t of the pair's sequence, CTA `cta` of it
+  const int cta = PAIR ? static_cast<int>(cluster_ctarank()) : 0;
+  const bool leader = cta == 0;
+  const int first_tile = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int tile_step = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
@@ -419,7 +463,8 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 32 * Roles<KIND>::kEpiWarps);
+      // the even CTA's MMA waits for the epilogues of both CTAs of a pair
+      mbar_init(&tempty[a], 32 * Roles<KIND>::kEpiWarps * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -434,8 +479,13 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     if (KIND == kWgrad) tma_prefetch_desc(&maps.b2);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(s_tmem, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(s_tmem, kTmemCols);
+      tmem_relinquish();
+    }
   }
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = p.offsets[e];
   __syncthreads();
@@ -461,7 +511,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       int v = 0;
       if (s < E) {
         const int e = s_order[s];
-        v = tiles_of_expert<KIND, BN>(static_cast<int>(s_off[e + 1] - s_off[e]), d, f);
+        v = tiles_of_expert<KIND, BN, PAIR>(static_cast<int>(s_off[e + 1] - s_off[e]), d, f);
       }
       int inc = v;
 #pragma unroll
@@ -479,6 +529,8 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  // both CTAs of a pair have their barriers initialised before either signals the other's
+  if (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int total = *s_total;
@@ -489,16 +541,22 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // last load issued on full[s], and its phase
-    for (int tile = blockIdx.x; tile < total && !*s_abort; tile += gridDim.x) {
-      const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
+    // loads of both CTAs of a pair complete on the even CTA's full barriers
+    const uint32_t full_leader = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
+    for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step) {
+      const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
       for (int kb = 0; kb < nk; ++kb) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, kWaitLimit)) break;
         uint8_t* a_dst = sA + stage * Tr::A_BYTES;
         uint8_t* b_dst = sB + stage * Tr::B_BYTES;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[stage], Tr::STAGE_TX);
-          issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
+          if (leader) mbar_arrive_expect_tx(&full[stage], Tr::STAGE_TX);
+          if (PAIR)
+            issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst,
+                                       full_leader + 8u * static_cast<uint32_t>(stage));
+          else
+            issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -508,20 +566,21 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         }
       }
     }
-    if (*s_abort) {
-      // leave no copy in flight into shared memory this CTA is about to free
+    if (*s_abort && leader) {
+      // leave no copy in flight into shared memory that is about to be freed
+      // (a pair's loads all count on the even CTA's barriers)
       volatile int never = 0;
       for (int s = 0; s < STAGES; ++s)
         if ((issued_mask >> s) & 1u) wait_bounded(&full[s], (issued_par >> s) & 1u, &never, kWaitLimit);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 && leader) {
     // ------------------------------------------------------- MMA issuer
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total && !*s_abort; tile += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
+    for (int tile = first_tile; ok && tile < total && !*s_abort; tile += tile_step, ++it) {
+      const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
@@ -566,9 +625,12 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
                                             : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bdesc = Tr::B_MN ? umma_desc_sw128(b_addr + kk * 2048, 8192, 1024)
                                             : umma_desc_sw128(b_addr + kk * 32, 16, 1024);
-            mma_bf16(dtm, adesc, bdesc, Tr::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            if (PAIR) mma_bf16_pair(dtm, adesc, bdesc, Tr::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else mma_bf16(dtm, adesc, bdesc, Tr::IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
-          mma_commit(&empty[stage]);
+          // the stage is free in both CTAs once these MMAs have read it
+          if (PAIR) mma_commit_pair_multicast(&empty[stage], 0x3);
+          else mma_commit(&empty[stage]);
         }
         __syncwarp();
         if (++stage == STAGES) {
@@ -577,24 +639,31 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         }
       }
       if (!ok) break;
-      if (lane == 0) mma_commit(&tfull[acc]);
+      if (lane == 0) {
+        if (PAIR) mma_commit_pair_multicast(&tfull[acc], 0x3);
+        else mma_commit(&tfull[acc]);
+      }
       __syncwarp();
     }
     // every MMA this thread issued has completed once `drain` flips
-    if (lane == 0) mma_commit(drain);
+    if (lane == 0) {
+      if (PAIR) mma_commit_pair_multicast(drain, 0x1);
+      else mma_commit(drain);
+    }
     __syncwarp();
     volatile int never = 0;
     wait_bounded(drain, 0, &never, kWaitLimit);
-  } else {
+  } else if (warp >= 2) {
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;
-    const int r = q * 32 + lane;
+    const int r = BM * cta + q * 32 + lane;  // row of the tile
     // with eight epilogue warps each handles half of the columns
     constexpr int kSplit = Roles<KIND>::kEpiWarps / 4;
     const int c0 = ((warp - 2) >> 2) * ((KIND == kFwdGateUp ? 128 : BN) / kSplit);
+    const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
     int it = 0;
-    for (int tile = blockIdx.x; tile < total && !*s_abort; tile += gridDim.x, ++it) {
-      const TileInfo ti = decode_tile<KIND, BN>(sched, tile, d, f);
+    for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step, ++it) {
+      const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       EpiCarry carry;
@@ -604,16 +673,21 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
       epilogue<KIND, BN>(p, ti, tacc, r, c0, carry);
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
+      else mbar_arrive(&tempty[acc]);
     }
   }
 
   // ------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still read its shared
+  // memory or write its TMEM
+  if (PAIR) cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem_base, kTmemCols);
+    else tmem_dealloc(tmem_base, kTmemCols);
   }
   if (threadIdx.x == 0 && *s_abort) raise_error(p.err, kErrTimeout);
 }
@@ -660,15 +734,41 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int KIND, int BN>
+template <int KIND, int BN, bool PAIR>
 static cudaError_t launch(const Maps& m, const Params& p, cudaStream_t s) {
-  using Tr = Traits<KIND, BN>;
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<KIND, BN>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+  using Tr = Traits<KIND, BN, PAIR>;
+  auto kern = grouped_gemm_kernel<KIND, BN, PAIR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(Tr::SMEM));
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<KIND, BN><<<sm_count(), Roles<KIND>::kThreads, Tr::SMEM, s>>>(m, p);
-  return cudaGetLastError();
+  if (!PAIR) {
+    kern<<<sm_count(), Roles<KIND>::kThreads, Tr::SMEM, s>>>(m, p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(sm_count() / 2 * 2));
+  cfg.blockDim = dim3(Roles<KIND>::kThreads);
+  cfg.dynamicSmemBytes = Tr::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // every pair must be resident at once: the tile sequence of a pair that
+  // starts late would finish a whole wave after the others
+  static int resident_pairs = 0;
+  if (resident_pairs == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(kern), &cfg) != cudaSuccess)
+      n = 0;
+    resident_pairs = n > 0 ? n : -1;
+  }
+  if (resident_pairs > 0 && static_cast<unsigned>(2 * resident_pairs) < cfg.gridDim.x)
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * resident_pairs));
+  return cudaLaunchKernelEx(&cfg, kern, m, p);
 }
 
 }  // namespace gg
@@ -689,14 +789,15 @@ cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   p.o0 = static_cast<bf16*>(a.h1);
   p.o1 = static_cast<bf16*>(a.h2);
   p.o2 = static_cast<bf16*>(a.a);
-  cudaError_t e = launch<kFwdGateUp, 256>(m1, p, s);
+  cudaError_t e = launch<kFwdGateUp, 256, true>(m1, p, s);
   if (e != cudaSuccess) return e;
   Maps m2{};
-  if (!make_map(&m2.a0, a.a, f, rows, f, 64, 128) || !make_map(&m2.b0, a.Wd, f, E * d, f, 64, 256))
+  // pairs: each CTA stages 128 of the tile's 256 Wd rows
+  if (!make_map(&m2.a0, a.a, f, rows, f, 64, 128) || !make_map(&m2.b0, a.Wd, f, E * d, f, 64, 128))
     return cudaErrorInvalidValue;
   p.o0 = static_cast<bf16*>(a.yp);
   p.o1 = p.o2 = nullptr;
-  return launch<kFwdDown, 256>(m2, p, s);
+  return launch<kFwdDown, 256, true>(m2, p, s);
 }
 
 static gg::Params bwd_params(const FfnBwdArgs& a) {
@@ -721,8 +822,8 @@ cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.i1 = static_cast<const bf16*>(a.h2);
   p.o0 = static_cast<bf16*>(a.dh1);
   p.o1 = static_cast<bf16*>(a.dh2);
-  cudaError_t e = (a.f % 256 == 0) ? launch<kBwdDgradDown, 256>(m1, p, s)
-                                   : launch<kBwdDgradDown, 128>(m1, p, s);
+  cudaError_t e = (a.f % 256 == 0) ? launch<kBwdDgradDown, 256, true>(m1, p, s)
+                                   : launch<kBwdDgradDown, 128, true>(m1, p, s);
   if (e != cudaSuccess) return e;
   // 2. dxp = dh1 Wg_e + dh2 Wu_e
   Maps m2{};
@@ -732,7 +833,7 @@ cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.i0 = p.i1 = nullptr;
   p.o0 = static_cast<bf16*>(a.dxp);
   p.o1 = nullptr;
-  return launch<kBwdDgradGateUp, 256>(m2, p, s);
+  return launch<kBwdDgradGateUp, 256, true>(m2, p, s);
 }
 
 cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
@@ -747,7 +848,33 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.w0 = a.dWg;
   p.w1 = a.dWu;
   p.w2 = a.dWd;
-  return launch<kWgrad, 256>(m3, p, s);
+  return launch<kWgrad, 256, false>(m3, p, s);
+}
+
+}  // namespace moe
+
+namespace moe {
+
+// One block waits on an mbarrier nothing arrives at, with the bounded wait
+// of the GEMM pipelines, and reports the time-out through the error word.
+__global__ void selftest_wait_timeout_kernel(unsigned* err, long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = sm100::wait_bounded(&bar, 0, &abort_flag, limit);
+    if (!ok) raise_error(err, kErrTimeout);
+  }
+}
+
+cudaError_t launch_selftest_wait_timeout(unsigned* err, long long limit, cudaStream_t s) {
+  selftest_wait_timeout_kernel<<<1, 32, 0, s>>>(err, limit);
+  return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -38,8 +38,9 @@ cudaError_t launch_combine_bwd(const void* dY, const void* yp, const float* w,
 cudaError_t launch_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dz,
                                const void* Wr, const int32_t* idx, int dtype, int64_t T, int d,
                                int E, int k, void* dX, cudaStream_t s);
-int router_bwd_splits(int64_t T, int d, int E);
-cudaError_t launch_router_bwd(const void* x, const float* dz, int dtype, int64_t T, int d, int E,
+int router_bwd_max_items(int64_t rows, int E);
+cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* pair_of_row,
+                              const int64_t* offsets, int dtype, int64_t rows, int d, int E, int k,
                               float* dWr, float* db, float* partial, cudaStream_t s);
 
 // grouped expert FFN (grouped_gemm_sm100.cu, grouped_simt.cu)
@@ -62,6 +63,7 @@ struct FfnBwdArgs {
   unsigned* err;
 };
 
+cudaError_t launch_selftest_wait_timeout(unsigned* err, long long limit, cudaStream_t s);
 cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 2 launches
 cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 1 launch

@@ -82,7 +82,7 @@ class MoELayer:
             "route": N._ws(N.moe_route_workspace_bytes(T, E), dev),
             "ffn_fwd": N._ws(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt), dev),
             "ffn_bwd": N._ws(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt), dev),
-            "router_bwd": N._ws(N.moe_router_bwd_workspace_bytes(T, d, E), dev),
+            "router_bwd": N._ws(N.moe_router_bwd_workspace_bytes(P, d, E), dev),
         }
         self.max_tokens = T
 
@@ -103,9 +103,10 @@ class MoELayer:
             ro[n] = r[n][:P]
         return v, ro
 
-    def forward(self, x: torch.Tensor, stream=None, mark=None) -> torch.Tensor:
-        """Y = layer(x). `mark(name)`, if given, is called after each C call
-        (the benchmark records CUDA events there)."""
+    def forward(self, x: torch.Tensor, stream=None, mark=None, out=None) -> torch.Tensor:
+        """Y = layer(x), written to `out` if given (else to a layer buffer).
+        `mark(name)`, if given, is called after each C call (the benchmark
+        records CUDA events there)."""
         mark = mark or _no_mark
         T = x.shape[0]
         self.reserve(T)
@@ -122,12 +123,14 @@ class MoELayer:
         N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"],
                               {n: v[n] for n in ("h1", "h2", "a", "yp")}, self.ws["ffn_fwd"], stream)
         mark("grouped_ffn_fwd")
-        N.moe_unpermute_combine(v["yp"], r["topk_w"], r["row_of_pair"], v["Y"], stream)
+        Y = v["Y"] if out is None else out
+        N.moe_unpermute_combine(v["yp"], r["topk_w"], r["row_of_pair"], Y, stream)
         mark("unpermute_combine")
-        return v["Y"]
+        return Y
 
-    def backward(self, dY: torch.Tensor, stream=None, mark=None) -> torch.Tensor:
-        """dX for upstream gradient dY of the last forward; dW += (fp32)."""
+    def backward(self, dY: torch.Tensor, stream=None, mark=None, out=None) -> torch.Tensor:
+        """dX for upstream gradient dY of the last forward (written to `out`
+        if given); dW += (fp32)."""
         mark = mark or _no_mark
         T = self.T
         v, r = self.v, self.r
@@ -142,12 +145,14 @@ class MoELayer:
         N.moe_grouped_ffn_wgrad(v["xp"], v["a"], v["dyp"], v["dh1"], v["dh2"], r["offsets"], g["dWg"],
                                 g["dWu"], g["dWd"], self.ws["ffn_bwd"], stream)
         mark("grouped_ffn_wgrad")
+        dX = v["dX"] if out is None else out
         N.moe_permute_bwd(v["dxp"], r["row_of_pair"], v["dlogits"], self.Wr, r["topk_idx"], T, self.k,
-                          v["dX"], stream)
+                          dX, stream)
         mark("permute_bwd")
-        N.moe_router_bwd(self.x, v["dlogits"], g["dWr"], g["db"], self.ws["router_bwd"], stream)
+        N.moe_router_bwd(v["xp"], v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"], g["db"],
+                         self.ws["router_bwd"], stream)
         mark("router_bwd")
-        return v["dX"]
+        return dX
 
     def device_errors(self) -> int:
         """Synchronises and returns (and clears) the device error words."""

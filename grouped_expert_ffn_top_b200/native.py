@@ -47,6 +47,7 @@ _SIGNATURES = {
     "moe_last_error": ([], ctypes.c_char_p),
     "moe_version": ([], _i),
     "moe_launch_count": ([], _i64),
+    "moe_selftest_wait_timeout": ([_p, ctypes.c_longlong, _p], _i),
     "moe_get_error": ([_p, _p], _i),
     "moe_router_logits": ([_p, _p, _p, _i, _i64, _i, _i, _p, _p], _i),
     "moe_route_workspace_bytes": ([_i64, _i], _sz),
@@ -64,7 +65,7 @@ _SIGNATURES = {
     "moe_grouped_ffn_wgrad": ([_p] * 5 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
     "moe_permute_bwd": ([_p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p], _i),
     "moe_router_bwd_workspace_bytes": ([_i64, _i, _i], _sz),
-    "moe_router_bwd": ([_p, _p, _i, _i64, _i, _i, _p, _p, _p, _sz, _p], _i),
+    "moe_router_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p, _p, _sz, _p], _i),
 }
 
 
@@ -296,15 +297,16 @@ def moe_permute_bwd(dxp, row_of_pair, dlogits, Wr, topk_idx, T: int, k: int, dX=
     return dX
 
 
-def moe_router_bwd_workspace_bytes(T, d, E) -> int:
-    return lib().moe_router_bwd_workspace_bytes(T, d, E)
+def moe_router_bwd_workspace_bytes(rows, d, E) -> int:
+    return lib().moe_router_bwd_workspace_bytes(rows, d, E)
 
 
-def moe_router_bwd(x, dlogits, dWr, db, ws=None, stream=None):
-    _contig(x, dlogits, dWr, db)
-    T, d = x.shape
-    E = dlogits.shape[1]
+def moe_router_bwd(xp, dlogits, pair_of_row, expert_offsets, k: int, dWr, db, ws=None, stream=None):
+    _contig(xp, dlogits, pair_of_row, expert_offsets, dWr, db)
+    rows, d = xp.shape
+    T, E = dlogits.shape
     if ws is None:
-        ws = _ws(moe_router_bwd_workspace_bytes(T, d, E), x.device)
-    _check(lib().moe_router_bwd(_ptr(x), _ptr(dlogits), _dt(x), T, d, E, _ptr(dWr), _ptr(db), _ptr(ws),
-                                ws.numel(), _stream(stream)), "moe_router_bwd")
+        ws = _ws(moe_router_bwd_workspace_bytes(rows, d, E), xp.device)
+    _check(lib().moe_router_bwd(_ptr(xp), _ptr(dlogits), _ptr(pair_of_row), _ptr(expert_offsets),
+                                _dt(xp), T, d, E, k, _ptr(dWr), _ptr(db), _ptr(ws), ws.numel(),
+                                _stream(stream)), "moe_router_bwd")

@@ -92,6 +92,14 @@ MOE_API int moe_version(void);
  * library's launches in it. */
 MOE_API int64_t moe_launch_count(void);
 
+/* Self-test of the kernels' failure detection: launches one block that
+ * waits on an mbarrier nothing ever arrives at, with the same bounded wait
+ * the grouped GEMMs use, giving up after `limit_cycles` SM cycles (clamped to
+ * [1e3, 4e9]). It then raises MOE_DEVERR_TIMEOUT in the ws error word and
+ * returns normally, so the CUDA context stays usable; moe_get_error(ws)
+ * reports it. ws: a zeroed workspace of at least 256 bytes. */
+MOE_API int moe_selftest_wait_timeout(void* ws, long long limit_cycles, cudaStream_t stream);
+
 /* Synchronises `stream`, returns the device error word accumulated in `ws`
  * by the calls that used it since the last moe_get_error (0 = no error), and
  * clears it. Returns MOE_ERR_CUDA (< 0) if the synchronisation fails. */
@@ -283,15 +291,26 @@ MOE_API int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const f
                     const void* Wr, const int32_t* topk_idx, int dtype, int64_t T, int d,
                     int E, int k, void* dX, cudaStream_t stream);
 
-/* Workspace of moe_router_bwd, in bytes. */
-MOE_API size_t moe_router_bwd_workspace_bytes(int64_t T, int d, int E);
+/* Workspace of moe_router_bwd, in bytes (rows = T*k). */
+MOE_API size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E);
 
 /* Router weight gradients (accumulated, fp32, deterministic order):
  *   dWr[e, :] += sum_t dlogits[t, e] x[t, :];   db[e] += sum_t dlogits[t, e]
- *   x [T, d] dtype; dlogits [T, E] fp32; dWr [E, d] fp32; db [E] fp32 (may be
- *   NULL). */
-MOE_API int moe_router_bwd(const void* x, const float* dlogits, int dtype, int64_t T, int d, int E,
-                   float* dWr, float* db, void* ws, size_t ws_bytes, cudaStream_t stream);
+ * (router backward of z = x Wr^T + b). The sums run over the dispatch rows
+ * instead of all tokens: expert e's rows [expert_offsets[e],
+ * expert_offsets[e+1]) hold exactly the tokens that selected e, and xp holds
+ * their x rows, so
+ *   dWr[e, :] += sum_{r in e} dlogits[pair_of_row[r] / k, e] xp[r, :].
+ * This equals the sum over all tokens when dlogits is zero off the selection,
+ * which moe_route_bwd guarantees; it reads xp once instead of computing a
+ * T x E x d product.
+ *   xp [T*k, d] dtype (moe_permute's output); dlogits [T, E] fp32;
+ *   pair_of_row [T*k], expert_offsets [E+1] (moe_route's outputs);
+ *   dWr [E, d] fp32 (+=); db [E] fp32 (+=, may be NULL). */
+MOE_API int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_row,
+                           const int64_t* expert_offsets, int dtype, int64_t T, int d, int E,
+                           int k, float* dWr, float* db, void* ws, size_t ws_bytes,
+                           cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -58,7 +58,7 @@ def test_workspace_sizes(L):
     assert big >= 256 + 2 * 4 * (32768 // 256) * 64
     assert L.moe_route_workspace_bytes(-1, 8) == 0
     assert L.moe_grouped_ffn_bwd_workspace_bytes(1000, 8, 256, 384, N.MOE_BF16) >= 2 * 1000 * 384 * 2
-    assert L.moe_router_bwd_workspace_bytes(4096, 1024, 8) >= 256 + 4 * 8 * 1025
+    assert L.moe_router_bwd_workspace_bytes(8192, 1024, 8) >= 256 + 4 * (8192 // 256 + 8) * 1025
 
 
 null = ctypes.c_void_p(0)
@@ -100,4 +100,7 @@ def test_row_pass_argument_errors(L):
     assert L.moe_permute_bwd(null, null, null, null, null, N.MOE_BF16, 4, 128, 2, 3, null, null) == \
         N.MOE_ERR_INVALID_ARG  # k > E
     assert L.moe_route_bwd(null, null, null, 4, 8, 9, null, null) == N.MOE_ERR_INVALID_ARG
-    assert L.moe_router_bwd(null, null, N.MOE_BF16, 0, 128, 8, null, null, null, 0, null) == N.MOE_OK
+    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 0, 128, 8, 2, null, null, null, 0,
+                            null) == N.MOE_OK
+    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 4, 128, 8, 9, null, null, null, 0,
+                            null) == N.MOE_ERR_INVALID_ARG

@@ -204,6 +204,22 @@ def test_all_tokens_on_one_expert():
         assert_close(n, layer.grads[n], bw[n], 2e-2)
 
 
+# ----------------------------------------------------- failure detection
+
+def test_bounded_wait_times_out_and_leaves_the_context_usable():
+    """A wait on a barrier nothing arrives at gives up, raises the time-out
+    bit in the error word, and the next calls still work."""
+    ws = N._ws(256, DEV)
+    rc = N.lib().moe_selftest_wait_timeout(N._ptr(ws), 2_000_000, N._stream(None))
+    assert rc == N.MOE_OK
+    assert N.moe_get_error(ws) == N.MOE_DEVERR_TIMEOUT
+    assert N.moe_get_error(ws) == 0
+    z = workloads.make_logits(100, 8, device=DEV, seed=1)
+    out = N.moe_route(z, 2)
+    idx, _, _ = oracle.route(z.double().cpu().numpy(), 2)
+    assert np.array_equal(to_np(out["topk_idx"]), idx)
+
+
 # ------------------------------------------------------- argument errors
 
 def test_rejected_calls_report_errors_and_launch_nothing():
