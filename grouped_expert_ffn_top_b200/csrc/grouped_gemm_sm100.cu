@@ -899,8 +899,9 @@ cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.i1 = static_cast<const bf16*>(a.h2);
   p.o0 = static_cast<bf16*>(a.dh1);
   p.o1 = static_cast<bf16*>(a.dh2);
-  cudaError_t e = (a.f % 256 == 0) ? launch<kBwdDgradDown, 256, true>(m1, p, s)
-                                   : launch<kBwdDgradDown, 128, true>(m1, p, s);
+  // 256-wide tiles even when f is not a multiple of 256 (a half-empty edge
+  // tile costs less than the narrower MMA everywhere else)
+  cudaError_t e = launch<kBwdDgradDown, 256, true>(m1, p, s);
   if (e != cudaSuccess) return e;
   // 2. dxp = dh1 Wg_e + dh2 Wu_e
   Maps m2{};
