@@ -86,9 +86,6 @@ struct Traits {
   static constexpr uint32_t B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;    // per CTA
   static constexpr uint32_t STAGE_TX = (A_BYTES + B_BYTES) * (PAIR ? 2 : 1);  // all CTAs
   static constexpr uint32_t IDESC = umma_idesc_bf16(TM, BN, A_MN, B_MN);
-  // a pair's ragged-K tail block: each CTA zeroes the rows past the expert's
-  // end in its own stage; the odd CTA then signals the even CTA's MMA warp
-  static constexpr bool PAIR_TAIL = PAIR && KIND == kWgrad;
   // N extent of one output tile (gate/up: 128 f columns, each with its gate
   // and up accumulator, together the MMA's N = 256)
   static constexpr int NTILE = KIND == kFwdGateUp ? 128 : BN;
@@ -261,23 +258,6 @@ __device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& 
     for (int j = 0; j < HALF / 64; ++j)
       tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, r);
   }
-}
-
-// The ragged-K tail block of a pair's wgrad tile, loaded by one CTA into its
-// own stage with a single-CTA TMA counted on its own barrier `bar`.
-template <int BN>
-__device__ __forceinline__ void issue_wgrad_tail_local(const Maps& m, const TileInfo& ti, int kb,
-                                                       int cta, uint8_t* a_dst, uint8_t* b_dst,
-                                                       uint64_t* bar) {
-  constexpr int HALF = BN / 2;
-  const CUtensorMap* am = ti.prod == 2 ? &m.a1 : &m.a0;
-  const CUtensorMap* bm = ti.prod == 0 ? &m.b0 : (ti.prod == 1 ? &m.b1 : &m.b2);
-  const int r = ti.row0 + kb * BK;
-  const int mm = ti.m0 + BM * cta;
-  tma_load_2d(a_dst, am, bar, mm, r);
-  tma_load_2d(a_dst + 8192, am, bar, mm + 64, r);
-#pragma unroll
-  for (int j = 0; j < HALF / 64; ++j) tma_load_2d(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, r);
 }
 
 __device__ __forceinline__ uint4 pack8_bf16(const float* v) {
@@ -453,6 +433,18 @@ __device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, ui
   }
 }
 
+// One K16 step of a stage: MMA of the stage's A and B at K offset 16 * kk.
+template <typename Tr, bool PAIR>
+__device__ __forceinline__ void issue_mma(uint32_t dtm, uint32_t a_addr, uint32_t b_addr, int kk,
+                                          uint32_t accumulate) {
+  const uint64_t adesc = Tr::A_MN ? umma_desc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                  : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
+  const uint64_t bdesc = Tr::B_MN ? umma_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                  : umma_desc_sw128(b_addr + kk * 32, 16, 1024);
+  if (PAIR) mma_bf16_pair(dtm, adesc, bdesc, Tr::IDESC, accumulate);
+  else mma_bf16(dtm, adesc, bdesc, Tr::IDESC, accumulate);
+}
+
 template <int KIND, int BN, bool PAIR>
 __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
@@ -469,9 +461,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* aux = drain + 1;        // a pair's ragged-K tail loads (this CTA's bytes only)
-  uint64_t* tailready = aux + 1;    // [STAGES] the odd CTA's tail stage is zeroed
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(tailready + STAGES);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort) + 1;
   int64_t* s_off = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(bars) + Tr::BAR_BYTES);
@@ -492,9 +482,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&tailready[s], 1);
     }
-    mbar_init(aux, 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       // the even CTA's MMA waits for the epilogues of both CTAs of a pair
@@ -573,12 +561,10 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     int stage = 0;
-    uint32_t phase = 0, aux_phase = 0;
-    bool aux_pending = false;
+    uint32_t phase = 0;
     uint32_t issued_mask = 0, issued_par = 0;  // last load issued on full[s], and its phase
     // loads of both CTAs of a pair complete on the even CTA's full barriers
     const uint32_t full_leader = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
-    const uint32_t tailready_leader = Tr::PAIR_TAIL ? mapa_shared(smem_u32(tailready), 0) : 0u;
     for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step) {
       const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
@@ -587,44 +573,16 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         uint8_t* a_dst = sA + stage * Tr::A_BYTES;
         uint8_t* b_dst = sB + stage * Tr::B_BYTES;
         const uint32_t full_addr = full_leader + 8u * static_cast<uint32_t>(stage);
-        if (Tr::PAIR_TAIL && (kb + 1) * BK > ti.rows) {
-          // ragged-K tail of a pair: this CTA loads its part on its own
-          // barrier, zeroes the rows past the expert's end (they belong to the
-          // next expert or lie past the tensor), then the even CTA completes
-          // its full barrier and the odd CTA its tail-ready barrier
-          if (lane == 0) {
-            mbar_arrive_expect_tx(aux, Tr::A_BYTES + Tr::B_BYTES);
-            issue_wgrad_tail_local<BN>(maps, ti, kb, cta, a_dst, b_dst, aux);
+        if (lane == 0) {
+          if (leader) mbar_arrive_expect_tx(&full[stage], Tr::STAGE_TX);
+          if (PAIR) {
+            issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst, full_addr);
+          } else {
+            issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
           }
-          aux_pending = true;
-          if (!wait_bounded(aux, aux_phase, s_abort, kWaitLimit)) break;
-          aux_pending = false;
-          aux_phase ^= 1u;
-          const int valid = ti.rows - kb * BK;
-          const int chunks = (BK - valid) * 8;  // 16-byte chunks per 64-column box
-          const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          for (int box = 0; box < 2 + BN / 128; ++box) {
-            uint8_t* base = (box < 2 ? a_dst + box * 8192 : b_dst + (box - 2) * 8192) + valid * 128;
-            for (int c = lane; c < chunks; c += 32) reinterpret_cast<uint4*>(base)[c] = z;
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if (leader) mbar_arrive(&full[stage]);
-            else mbar_arrive_cluster(tailready_leader + 8u * static_cast<uint32_t>(stage));
-          }
-        } else {
-          if (lane == 0) {
-            if (leader) mbar_arrive_expect_tx(&full[stage], Tr::STAGE_TX);
-            if (PAIR) {
-              issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst, full_addr);
-            } else {
-              issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
-            }
-          }
-          issued_mask |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         }
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1u;
@@ -638,13 +596,11 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       if (leader)
         for (int s = 0; s < STAGES; ++s)
           if ((issued_mask >> s) & 1u) wait_bounded(&full[s], (issued_par >> s) & 1u, &never, kWaitLimit);
-      if (aux_pending) wait_bounded(aux, aux_phase, &never, kWaitLimit);
     }
   } else if (warp == 1 && leader) {
     // ------------------------------------------------------- MMA issuer
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t tail_par = 0;  // per stage: parity of its next tail-ready phase
     int it = 0;
     bool ok = true;
     for (int tile = first_tile; ok && tile < total && !*s_abort; tile += tile_step, ++it) {
@@ -661,15 +617,6 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
           break;
         }
         tc_fence_after();
-        if (Tr::PAIR_TAIL && (kb + 1) * BK > ti.rows) {
-          // the odd CTA's half of this tail stage must be zeroed as well
-          if (!wait_bounded(&tailready[stage], (tail_par >> stage) & 1u, s_abort, kWaitLimit)) {
-            ok = false;
-            break;
-          }
-          tail_par ^= 1u << stage;
-          tc_fence_after();
-        }
         int ksteps = BK / 16;
         if (KIND == kWgrad && (kb + 1) * BK > ti.rows) {
           // ragged-K tail: rows past the expert's end belong to the next
@@ -679,31 +626,40 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
           const int valid = ti.rows - kb * BK;
           ksteps = (valid + 15) / 16;
           const int zrows = ksteps * 16 - valid;
-          if (!PAIR && zrows > 0) {  // a pair's producers zeroed their own stages
-            uint8_t* a_st = sA + stage * Tr::A_BYTES;
-            uint8_t* b_st = sB + stage * Tr::B_BYTES;
-            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-            const int chunks = zrows * 8;  // 16-byte chunks per 64-column box
-            for (int box = 0; box < 2 + BN / 64; ++box) {
-              uint8_t* base = (box < 2 ? a_st + box * 8192 : b_st + (box - 2) * 8192) + valid * 128;
-              for (int c = lane; c < chunks; c += 32) reinterpret_cast<uint4*>(base)[c] = z;
+          if (zrows > 0) {
+            // each 64-column box holds one 128-byte row per K row, so the rows
+            // to clear are one contiguous range per box; a pair's MMA also
+            // reads the odd CTA's stage, which this warp clears through
+            // distributed shared memory
+            const uint32_t a_st = smem_u32(sA + stage * Tr::A_BYTES);
+            const uint32_t b_st = smem_u32(sB + stage * Tr::B_BYTES);
+            const int chunks = zrows * 8;  // 16-byte chunks per box
+            constexpr int kBoxes = 2 + static_cast<int>(Tr::B_BYTES / 8192);
+            for (int peer = 0; peer < (PAIR ? 2 : 1); ++peer) {
+              for (int box = 0; box < kBoxes; ++box) {
+                uint32_t base = (box < 2 ? a_st + box * 8192 : b_st + (box - 2) * 8192) + valid * 128;
+                if (PAIR) base = mapa_shared(base, static_cast<uint32_t>(peer));
+                for (int c = lane; c < chunks; c += 32) st_cluster_zero16(base + 16u * c);
+              }
             }
-            fence_proxy_async_smem();
+            if (PAIR) fence_proxy_async_cluster();
+            else fence_proxy_async_smem();
           }
           __syncwarp();
         }
         if (lane == 0) {
           const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
+          // A full block issues its four MMAs as straight-line code: a loop
+          // with a run-time bound between them leaves the tensor pipe idle
+          // between instructions. Only a ragged wgrad tail takes the loop.
+          if (ksteps == BK / 16) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            if (kk >= ksteps) break;
-            const uint64_t adesc = Tr::A_MN ? umma_desc_sw128(a_addr + kk * 2048, 8192, 1024)
-                                            : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
-            const uint64_t bdesc = Tr::B_MN ? umma_desc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                            : umma_desc_sw128(b_addr + kk * 32, 16, 1024);
-            if (PAIR) mma_bf16_pair(dtm, adesc, bdesc, Tr::IDESC, (kb | kk) != 0 ? 1u : 0u);
-            else mma_bf16(dtm, adesc, bdesc, Tr::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, (kb | kk) != 0 ? 1u : 0u);
+          } else {
+            for (int kk = 0; kk < ksteps; ++kk)
+              issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, (kb | kk) != 0 ? 1u : 0u);
           }
           // the stage is free in both CTAs once these MMAs have read it
           if (PAIR) mma_commit_pair_multicast(&empty[stage], 0x3);
@@ -926,8 +882,9 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.w0 = a.dWg;
   p.w1 = a.dWu;
   p.w2 = a.dWd;
-  // one-CTA tiles: with the pair tail handshake, CTA pairs measured no faster here
-  return launch<kWgrad, 256, false>(m3, p, s);
+  // CTA pairs: six stages of 32 KB per CTA hide more load latency than four
+  // of 48 KB
+  return launch<kWgrad, 256, true>(m3, p, s);
 }
 
 }  // namespace moe

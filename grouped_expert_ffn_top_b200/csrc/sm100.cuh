@@ -171,6 +171,18 @@ __device__ __forceinline__ void cluster_sync_all() {
 
 // Arrive on an mbarrier given by its shared::cluster address (possibly in
 // the peer CTA).
+// 16 zero bytes at a shared::cluster address (this CTA's or a peer's).
+__device__ __forceinline__ void st_cluster_zero16(uint32_t cluster_addr) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(cluster_addr), "r"(0u)
+               : "memory");
+}
+
+// Orders this thread's generic-proxy writes to shared::cluster memory before
+// later async-proxy reads of it (a peer CTA's MMA operands).
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");

@@ -204,6 +204,41 @@ def test_all_tokens_on_one_expert():
         assert_close(n, layer.grads[n], bw[n], 2e-2)
 
 
+def test_long_ragged_weight_gradient_is_exact_and_reproducible():
+    """Two experts of 4500 rows each: every weight-gradient tile runs 70 full
+    64-row K blocks and a tail of 20 rows, ragged inside a 16-row MMA step.
+    Full dW against the oracle, then the same backward again from zero must
+    give bitwise the same dW."""
+    T, d, E, k, f = 4500, 192, 3, 2, 256
+    w = workloads.custom("chunks", T, d, E, k, f, bias="zero")
+    p = workloads.make_params(w, device=DEV, seed=5)
+    p["b"][:] = 0.0
+    p["b"][2] = -1.0e4
+    bt = workloads.make_batch(w, device=DEV, seed=5)
+    layer = MoELayer(p, k, 1, max_tokens=T)
+    layer.forward(bt["x"])
+    layer.backward(bt["dY"])
+    torch.cuda.synchronize()
+    assert layer.device_errors() == 0
+    counts = to_np(layer.r["counts"])
+    assert counts.tolist() == [T, T, 0]
+    P = _np_params(p)
+    x64 = to_np(bt["x"]).astype(np.float64)
+    fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k)
+    bw = oracle.layer_backward(fw, x64, to_np(bt["dY"]).astype(np.float64), P["Wr"], P["Wg"], P["Wu"],
+                               P["Wd"], k)
+    first = {n: layer.grads[n].clone() for n in ("dWg", "dWu", "dWd")}
+    for n in first:
+        assert_close(n, first[n], bw[n], 2e-2)
+        assert not first[n][2].any()
+    layer.zero_grad()
+    layer.backward(bt["dY"])
+    torch.cuda.synchronize()
+    assert layer.device_errors() == 0
+    for n in first:
+        assert torch.equal(layer.grads[n], first[n]), n
+
+
 # ----------------------------------------------------- failure detection
 
 def test_bounded_wait_times_out_and_leaves_the_context_usable():
