@@ -39,7 +39,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
 template <int KIND>
 struct Roles {
-  static constexpr int kEpiWarps = (KIND == 2 || KIND == 4) ? 8 : 4;  // dgrad-down, wgrad
+  static constexpr int kEpiWarps = KIND == 4 ? 8 : 4;  // wgrad: eight
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
 };
 constexpr int kMaxE = MOE_MAX_EXPERTS;
@@ -56,6 +56,7 @@ enum Kind : int {
 
 struct Maps {
   CUtensorMap a0, a1, b0, b1, b2;
+  CUtensorMap o0, o1, o2;  // TMA-stored outputs (32 x 32 boxes, 64-byte swizzle)
 };
 
 struct Params {
@@ -81,7 +82,19 @@ struct Traits {
   static constexpr bool A_MN = KIND == kWgrad;
   static constexpr bool B_MN = KIND == kBwdDgradDown || KIND == kBwdDgradGateUp || KIND == kWgrad;
   static constexpr int TM = PAIR ? 2 * BM : BM;  // rows of one tile
-  static constexpr int STAGES = (PAIR || BN != 256) ? 6 : 4;
+  // Kinds whose epilogue writes bf16 tiles through shared memory with TMA
+  // stores: per epilogue warp, two buffers of a 32 x 32 box per output tensor
+  // (the SwiGLU backward also loads h1 / h2 into them and works in place).
+  static constexpr bool EPI_TMA = KIND == kFwdGateUp || KIND == kFwdDown || KIND == kBwdDgradGateUp;
+  static constexpr int EPI_TENSORS = KIND == kFwdGateUp ? 3 : (KIND == kBwdDgradDown ? 2 : 1);
+  static constexpr uint32_t EPI_BOX_BYTES = 32 * 32 * 2;
+  static constexpr uint32_t EPI_WARP_BYTES =
+      (EPI_TMA || KIND == kBwdDgradDown) ? 2 * EPI_TENSORS * EPI_BOX_BYTES : 0;
+  static constexpr uint32_t EPI_BYTES = EPI_WARP_BYTES * Roles<KIND>::kEpiWarps;
+  // pipeline stages: as many as fit beside the epilogue buffers and the
+  // schedule of up to 1024 experts
+  static constexpr int STAGES =
+      (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? 5 : ((PAIR || BN != 256) ? 6 : 4);
   static constexpr uint32_t A_BYTES = BM * BK * 2;                      // per CTA
   static constexpr uint32_t B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;    // per CTA
   static constexpr uint32_t STAGE_TX = (A_BYTES + B_BYTES) * (PAIR ? 2 : 1);  // all CTAs
@@ -90,9 +103,14 @@ struct Traits {
   // and up accumulator, together the MMA's N = 256)
   static constexpr int NTILE = KIND == kFwdGateUp ? 128 : BN;
   static constexpr size_t BAR_BYTES = 256;
-  static constexpr size_t SCHED_BYTES = 8 * (kMaxE + 1) + 4 * (kMaxE + 1) + 4 * kMaxE;
-  static constexpr size_t SMEM =
-      1024 + STAGES * static_cast<size_t>(A_BYTES + B_BYTES) + BAR_BYTES + SCHED_BYTES;
+  // dynamic shared memory: alignment slack, stages, barriers, and the tile
+  // schedule (expert offsets, first tile and expert of each slot) for E experts
+  static constexpr size_t SMEM_FIXED =
+      1024 + STAGES * static_cast<size_t>(A_BYTES + B_BYTES) + EPI_BYTES + BAR_BYTES;
+  static constexpr size_t smem_bytes(int E) {
+    return SMEM_FIXED + 8 * static_cast<size_t>(E + 1) + 4 * static_cast<size_t>(E + 1) +
+           4 * static_cast<size_t>(E);
+  }
   static_assert(KIND != kFwdGateUp || BN == 256, "gate/up pairs two 128-column accumulators");
   static_assert(2 * BN <= static_cast<int>(kTmemCols), "two accumulators must fit in TMEM");
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
@@ -293,144 +311,217 @@ __device__ __forceinline__ void red_add_f32(float* addr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
-// h1 / h2 values of 32 columns of this thread's row, loaded one chunk ahead
-// of their use by the SwiGLU-backward epilogue.
-struct EpiCarry {
-  uint4 h1[4], h2[4];
-};
-
-__device__ __forceinline__ void load_h_chunk(const Params& p, int64_t off, EpiCarry& c) {
-  const uint4* a = reinterpret_cast<const uint4*>(p.i0 + off);
-  const uint4* b = reinterpret_cast<const uint4*>(p.i1 + off);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    c.h1[i] = __ldg(a + i);
-    c.h2[i] = __ldg(b + i);
-  }
-}
-
-// Work an epilogue thread starts before its accumulator is ready: the first
-// chunk of h1 / h2 goes to registers, the rest of the row to L2.
-template <int KIND, int BN>
-__device__ __forceinline__ void epilogue_prefetch(const Params& p, const TileInfo& ti, int r,
-                                                  int c0, EpiCarry& carry) {
-  if (KIND == kBwdDgradDown) {
-    const int cols = min(c0 + BN / 2, p.f - ti.n0);
-    if (r < ti.rows && c0 < cols) {
-      const int64_t off = (static_cast<int64_t>(ti.row0) + r) * p.f + ti.n0;
-      load_h_chunk(p, off + c0, carry);
-      for (int c = c0 + 64; c < cols; c += 64) {  // 64 bf16 = one 128-byte line
-        prefetch_l2(p.i0 + off + c);
-        prefetch_l2(p.i1 + off + c);
-      }
-    }
-  }
-}
-
-// Epilogue of one tile for this thread's accumulator row r, on the columns
-// [c0, c0 + W) of the accumulator, W = BN / (epilogue warps / 4) (the gate/up
-// kind: f columns [c0, c0 + 128 / split), each with its gate and up
-// accumulator).
-template <int KIND, int BN>
-__device__ __forceinline__ void epilogue(const Params& p, const TileInfo& ti, uint32_t tacc,
-                                         int r, int c0, EpiCarry& carry) {
+// Weight-gradient epilogue of one tile for this thread's accumulator row r,
+// on the columns [c0, c0 + BN / 2) of the accumulator.
+template <int BN>
+__device__ __forceinline__ void epilogue_wgrad(const Params& p, const TileInfo& ti, uint32_t tacc,
+                                               int r, int c0) {
+  // Accumulator row m, column n is element (n, m) of the [N, M] row-major
+  // output, so for each column the 32 lanes of a warp cover 32 consecutive
+  // floats: one coalesced 128-byte reduction per column. red.global.add is
+  // fire-and-forget (the add happens at L2), and each element receives
+  // exactly one add per call, so the result is deterministic.
   const int d = p.d, f = p.f;
+  const int M = ti.prod == 2 ? f : d;
+  const int Nn = ti.prod == 2 ? d : f;
+  const int m = ti.m0 + r;
+  const bool valid = m < M;
+  float* out = (ti.prod == 0 ? p.w0 : (ti.prod == 1 ? p.w1 : p.w2)) +
+               static_cast<int64_t>(ti.e) * d * f + m;
   uint32_t u[16];
-  float v[16];
-  if (KIND == kFwdGateUp) {
-    const bool valid = r < ti.rows;
-    const int64_t row = static_cast<int64_t>(ti.row0) + r;
-    for (int c = c0; c < c0 + 128 / (Roles<KIND>::kEpiWarps / 4); c += 16) {
-      uint32_t g[16];
-      tmem_ld16(tacc + c, g);
-      tmem_ld16(tacc + 128 + c, u);
-      tmem_ld_wait();
-      if (valid && ti.n0 + c < f) {
-        float h1[16], h2[16], a[16];
+  for (int c = c0; c < c0 + BN / 2; c += 16) {
+    tmem_ld16(tacc + c, u);
+    tmem_ld_wait();
+    if (valid && ti.n0 + c < Nn) {
+      float* q = out + static_cast<int64_t>(ti.n0 + c) * M;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          h1[i] = __uint_as_float(g[i]);
-          h2[i] = __uint_as_float(u[i]);
-          a[i] = silu_f(h1[i]) * h2[i];
-        }
-        const int64_t off = row * f + ti.n0 + c;
-        store16_bf16(p.o0 + off, h1);
-        store16_bf16(p.o1 + off, h2);
-        store16_bf16(p.o2 + off, a);
-      }
+      for (int i = 0; i < 16; ++i) red_add_f32(q + static_cast<int64_t>(i) * M, __uint_as_float(u[i]));
     }
-  } else if (KIND == kFwdDown || KIND == kBwdDgradGateUp) {
-    const bool valid = r < ti.rows;
-    const int64_t row = static_cast<int64_t>(ti.row0) + r;
-    for (int c = c0; c < c0 + BN / (Roles<KIND>::kEpiWarps / 4); c += 16) {
-      tmem_ld16(tacc + c, u);
-      tmem_ld_wait();
-      if (valid && ti.n0 + c < d) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(u[i]);
-        store16_bf16(p.o0 + row * d + ti.n0 + c, v);
-      }
-    }
-  } else if (KIND == kBwdDgradDown) {
-    // chunks of 32 columns; h1 / h2 of the next chunk load while this one
-    // is computed (the first chunk was loaded before the accumulator wait)
-    const bool valid = r < ti.rows;
-    const int64_t base = (static_cast<int64_t>(ti.row0) + r) * f + ti.n0;
-    const int cols = min(c0 + BN / 2, f - ti.n0);
-    for (int c = c0; c < c0 + BN / 2; c += 32) {
-      EpiCarry next;
-      if (valid && c + 32 < cols) load_h_chunk(p, base + c + 32, next);
-      uint32_t u2[16];
-      tmem_ld16(tacc + c, u);
-      tmem_ld16(tacc + c + 16, u2);
-      tmem_ld_wait();
-      if (valid && c < cols) {
-        float h1[32], h2[32], dh1[32], dh2[32];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          unpack8_bf16(carry.h1[i], h1 + 8 * i);
-          unpack8_bf16(carry.h2[i], h2 + 8 * i);
-        }
+  }
+}
+
+// Epilogue of the kinds that write bf16 tiles (gate/up: h1, h2, a; down: yp;
+// dgrad gate/up: dxp) for one warp: its 32 accumulator rows (tile rows
+// rbase .. rbase + 31), in chunks of 32 columns. Where all 32 rows lie inside
+// the expert, each chunk goes row by row into a 64-byte-swizzled shared
+// buffer and one lane stores the 32 x 32 box with TMA, so the warp issues no
+// scattered global stores (those stall the MMA warp's issue on the same SM).
+// Rows past the expert's end belong to the next expert, so a warp with fewer
+// valid rows stores its valid rows directly. Two buffers per tensor
+// alternate (`ebuf`); a buffer is rewritten once its store has read it.
+template <int KIND, int BN>
+__device__ __forceinline__ void epilogue_tma(const Params& p, const Maps& maps, const TileInfo& ti,
+                                             uint32_t tacc, int rbase, int lane, uint8_t* sbuf,
+                                             int& ebuf) {
+  constexpr int NT = KIND == kFwdGateUp ? 3 : 1;  // output tensors
+  constexpr int W = KIND == kFwdGateUp ? 128 : BN;  // output columns of the tile
+  constexpr uint32_t BOX = 32 * 32 * 2;
+  const int ncols = KIND == kFwdGateUp ? p.f : p.d;
+  const int valid = min(32, ti.rows - rbase);  // rows of this warp inside the expert
+  if (valid <= 0) return;
+  const bool full = valid == 32;
+  const int64_t row = static_cast<int64_t>(ti.row0) + rbase + lane;
+  const CUtensorMap* omap[3] = {&maps.o0, &maps.o1, &maps.o2};
+  bf16* optr[3] = {p.o0, p.o1, p.o2};
+  for (int c = 0; c < W; c += 32) {
+    if (ti.n0 + c >= ncols) break;
+    float o[NT][32];
+    {
+      uint32_t u0[16], u1[16];
+      tmem_ld16(tacc + c, u0);
+      tmem_ld16(tacc + c + 16, u1);
+      if (KIND == kFwdGateUp) {
+        uint32_t g0[16], g1[16];
+        tmem_ld16(tacc + 128 + c, g0);
+        tmem_ld16(tacc + 128 + c + 16, g1);
+        tmem_ld_wait();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float da = __uint_as_float(i < 16 ? u[i] : u2[i - 16]);
-          const float sg = sigmoid_f(h1[i]);
-          dh1[i] = da * h2[i] * sg * (1.0f + h1[i] * (1.0f - sg));
-          dh2[i] = da * h1[i] * sg;
+          const float h1 = __uint_as_float(i < 16 ? u0[i] : u1[i - 16]);
+          const float h2 = __uint_as_float(i < 16 ? g0[i] : g1[i - 16]);
+          o[0][i] = h1;
+          o[1 % NT][i] = h2;
+          o[2 % NT][i] = silu_f(h1) * h2;
         }
-        store16_bf16(p.o0 + base + c, dh1);
-        store16_bf16(p.o0 + base + c + 16, dh1 + 16);
-        store16_bf16(p.o1 + base + c, dh2);
-        store16_bf16(p.o1 + base + c + 16, dh2 + 16);
-      }
-      carry = next;
-    }
-  } else {  // kWgrad
-    // Accumulator row m, column n is element (n, m) of the [N, M] row-major
-    // output, so for each column the 32 lanes of a warp cover 32 consecutive
-    // floats: one coalesced 128-byte reduction per column. red.global.add is
-    // fire-and-forget (the add happens at L2), and each element receives
-    // exactly one add per call, so the result is deterministic.
-    const int M = ti.prod == 2 ? f : d;
-    const int Nn = ti.prod == 2 ? d : f;
-    const int m = ti.m0 + r;
-    const bool valid = m < M;
-    float* out = (ti.prod == 0 ? p.w0 : (ti.prod == 1 ? p.w1 : p.w2)) +
-                 static_cast<int64_t>(ti.e) * d * f + m;
-    for (int c = c0; c < c0 + BN / 2; c += 16) {
-      tmem_ld16(tacc + c, u);
-      tmem_ld_wait();
-      if (valid && ti.n0 + c < Nn) {
-        float* q = out + static_cast<int64_t>(ti.n0 + c) * M;
+      } else {
+        tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) red_add_f32(q + static_cast<int64_t>(i) * M, __uint_as_float(u[i]));
+        for (int i = 0; i < 32; ++i) o[0][i] = __uint_as_float(i < 16 ? u0[i] : u1[i - 16]);
+      }
+    }
+    if (full) {
+      uint8_t* b = sbuf + ebuf * NT * BOX;
+      // the store that used this buffer two chunks ago has read it
+      if (lane == 0) bulk_wait_group_read<1>();
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        // row `lane`: four 16-byte chunks, chunk j at (j ^ ((lane >> 1) & 3)),
+        // the TMA 64-byte swizzle of a 64-byte row
+        uint8_t* rowp = b + t * BOX + lane * 64;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(rowp + ((j ^ ((lane >> 1) & 3)) << 4)) = pack8_bf16(o[t] + 8 * j);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) tma_store_2d(omap[t], b + t * BOX, ti.n0 + c, ti.row0 + rbase);
+        bulk_commit_group();
+      }
+      ebuf ^= 1;
+    } else if (lane < valid) {
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        bf16* dst = optr[t] + row * ncols + ti.n0 + c;
+        store16_bf16(dst, o[t]);
+        store16_bf16(dst + 16, o[t] + 16);
       }
     }
   }
+}
+
+// SwiGLU-backward epilogue of the dgrad-down kind for one warp: its 32 rows
+// (tile rows rbase .. rbase + 31), all columns of the tile in chunks of 32.
+//   dh1 = da h2 s (1 + h1 (1 - s)),  dh2 = da h1 s,  s = sigmoid(h1)
+// One lane loads the chunk's h1 and h2 boxes with TMA into a 64-byte-swizzled
+// buffer pair, one chunk ahead (two pairs alternate; each completes on its own
+// barrier of this warp); each lane then turns its row of h1, h2 and da into
+// dh1, dh2 in place, and one lane stores both boxes with TMA. Rows past the
+// expert's end are loaded and computed but not stored: a warp with fewer
+// valid rows writes its valid rows directly. `lphase` holds the parity of the
+// next completion of each of the warp's two barriers. Returns false if a wait
+// gave up (the kernel is aborting); loads it issued have landed by then.
+template <int BN>
+__device__ __forceinline__ bool epilogue_swiglu_bwd(const Params& p, const Maps& maps,
+                                                    const TileInfo& ti, uint32_t tacc, int rbase,
+                                                    int lane, uint8_t* sbuf, uint64_t* lbar,
+                                                    uint32_t& lphase, volatile int* s_abort) {
+  constexpr uint32_t BOX = 32 * 32 * 2;
+  const int valid = min(32, ti.rows - rbase);
+  if (valid <= 0) return true;
+  const int nch = min(BN, p.f - ti.n0) / 32;
+  const int y = ti.row0 + rbase;
+  const int64_t row = static_cast<int64_t>(y) + lane;
+  // buffer pair b: h1 (then dh1) at sbuf + 2 b BOX, h2 (then dh2) after it
+  auto load = [&](int ch, int b) {
+    if (lane == 0) {
+      bulk_wait_group_read<0>();  // earlier stores from these buffers have read them
+      mbar_arrive_expect_tx(&lbar[b], 2 * BOX);
+      tma_load_2d(sbuf + 2 * b * BOX, &maps.a1, &lbar[b], ti.n0 + 32 * ch, y);
+      tma_load_2d(sbuf + 2 * b * BOX + BOX, &maps.b1, &lbar[b], ti.n0 + 32 * ch, y);
+    }
+    __syncwarp();
+  };
+  uint32_t pend = 1u;  // buffer pairs with a load in flight
+  load(0, 0);
+  bool ok = true;
+  for (int ch = 0; ch < nch; ++ch) {
+    const int b = ch & 1;
+    if (ch + 1 < nch) {
+      load(ch + 1, b ^ 1);
+      pend |= 1u << (b ^ 1);
+    }
+    uint32_t u0[16], u1[16];
+    tmem_ld16(tacc + 32 * ch, u0);
+    tmem_ld16(tacc + 32 * ch + 16, u1);
+    tmem_ld_wait();
+    if (!wait_bounded(&lbar[b], (lphase >> b) & 1u, s_abort, kWaitLimit)) {
+      ok = false;
+      break;
+    }
+    lphase ^= 1u << b;
+    pend &= ~(1u << b);
+    uint8_t* r1 = sbuf + 2 * b * BOX + lane * 64;
+    uint8_t* r2 = r1 + BOX;
+    float dh1[32], dh2[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int off = (j ^ ((lane >> 1) & 3)) << 4;  // TMA 64-byte swizzle of a 64-byte row
+      float h1[8], h2[8];
+      unpack8_bf16(*reinterpret_cast<const uint4*>(r1 + off), h1);
+      unpack8_bf16(*reinterpret_cast<const uint4*>(r2 + off), h2);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int k = 8 * j + i;
+        const float da = __uint_as_float(k < 16 ? u0[k] : u1[k - 16]);
+        const float sg = sigmoid_f(h1[i]);
+        dh1[k] = da * h2[i] * sg * (1.0f + h1[i] * (1.0f - sg));
+        dh2[k] = da * h1[i] * sg;
+      }
+      *reinterpret_cast<uint4*>(r1 + off) = pack8_bf16(dh1 + 8 * j);
+      *reinterpret_cast<uint4*>(r2 + off) = pack8_bf16(dh2 + 8 * j);
+    }
+    if (valid == 32) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&maps.o0, sbuf + 2 * b * BOX, ti.n0 + 32 * ch, y);
+        tma_store_2d(&maps.o1, sbuf + 2 * b * BOX + BOX, ti.n0 + 32 * ch, y);
+        bulk_commit_group();
+      }
+    } else {
+      if (lane < valid) {
+        const int64_t off = row * p.f + ti.n0 + 32 * ch;
+        store16_bf16(p.o0 + off, dh1);
+        store16_bf16(p.o0 + off + 16, dh1 + 16);
+        store16_bf16(p.o1 + off, dh2);
+        store16_bf16(p.o1 + off + 16, dh2 + 16);
+      }
+      __syncwarp();
+    }
+  }
+  if (!ok) {
+    // leave no TMA copy in flight into this warp's buffers
+    volatile int never = 0;
+    for (int b = 0; b < 2; ++b)
+      if ((pend >> b) & 1u) {
+        wait_bounded(&lbar[b], (lphase >> b) & 1u, &never, kWaitLimit);
+        lphase ^= 1u << b;
+      }
+  }
+  return ok;
 }
 
 // One K16 step of a stage: MMA of the stage's A and B at K offset 16 * kk.
@@ -455,18 +546,20 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * Tr::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * Tr::B_BYTES);
+  uint8_t* sEpi = sB + STAGES * Tr::B_BYTES;  // 1024-aligned: stages are multiples of 1 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + Tr::EPI_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* lbar = drain + 1;  // [8] SwiGLU-backward epilogue loads: two per epilogue warp
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(lbar + 8);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort) + 1;
   int64_t* s_off = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(bars) + Tr::BAR_BYTES);
-  int* s_tstart = reinterpret_cast<int*>(s_off + kMaxE + 1);
-  int* s_order = s_tstart + kMaxE + 1;
+  int* s_tstart = reinterpret_cast<int*>(s_off + p.E + 1);
+  int* s_order = s_tstart + p.E + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -489,6 +582,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       mbar_init(&tempty[a], 32 * Roles<KIND>::kEpiWarps * (PAIR ? 2 : 1));
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&lbar[i], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -694,20 +788,35 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     constexpr int kSplit = Roles<KIND>::kEpiWarps / 4;
     const int c0 = ((warp - 2) >> 2) * ((KIND == kFwdGateUp ? 128 : BN) / kSplit);
     const uint32_t tempty_leader = PAIR ? mapa_shared(smem_u32(tempty), 0) : 0u;
+    int ebuf = 0;         // TMA-stored epilogues: staging buffer of the next 32-column chunk
+    uint32_t lphase = 0;  // SwiGLU-backward epilogue: parity of this warp's two load barriers
     int it = 0;
     for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step, ++it) {
       const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      EpiCarry carry;
-      epilogue_prefetch<KIND, BN>(p, ti, r, c0, carry);
       if (!wait_bounded(&tfull[acc], acc_phase, s_abort, kWaitLimit)) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-      epilogue<KIND, BN>(p, ti, tacc, r, c0, carry);
+      if constexpr (Tr::EPI_TMA) {
+        epilogue_tma<KIND, BN>(p, maps, ti, tacc, BM * cta + q * 32, lane,
+                               sEpi + (warp - 2) * Tr::EPI_WARP_BYTES, ebuf);
+      } else if constexpr (KIND == kBwdDgradDown) {
+        if (!epilogue_swiglu_bwd<BN>(p, maps, ti, tacc, BM * cta + q * 32, lane,
+                                     sEpi + (warp - 2) * Tr::EPI_WARP_BYTES, lbar + 2 * (warp - 2),
+                                     lphase, s_abort))
+          break;
+      } else {
+        epilogue_wgrad<BN>(p, ti, tacc, r, c0);
+      }
       tc_fence_before();
       if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
       else mbar_arrive(&tempty[acc]);
+    }
+    // this warp's TMA stores have finished before the CTA may exit
+    if (Tr::EPI_TMA || KIND == kBwdDgradDown) {
+      if (lane == 0) bulk_wait_group<0>();
+      __syncwarp();
     }
   }
 
@@ -746,9 +855,11 @@ static EncodeTiledFn encode_fn() {
 }
 
 // 2D bf16 tensor [outer, inner] (inner contiguous, row pitch `pitch` elements),
-// box [box_outer, box_inner], 128-byte swizzle, out-of-bounds reads as zero.
+// box [box_outer, box_inner], 128-byte swizzle unless given, out-of-bounds
+// reads as zero.
 static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
-                     uint64_t pitch, uint32_t box_inner, uint32_t box_outer) {
+                     uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+                     CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -756,8 +867,12 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Map of an epilogue's TMA boxes: [rows, cols] bf16, 32 x 32 boxes, 64-byte swizzle.
+static bool make_store_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows) {
+  return make_map(m, base, cols, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 static int sm_count() {
@@ -770,18 +885,20 @@ static int sm_count() {
 template <int KIND, int BN, bool PAIR>
 static cudaError_t launch(const Maps& m, const Params& p, cudaStream_t s) {
   using Tr = Traits<KIND, BN, PAIR>;
+  static_assert(Tr::smem_bytes(kMaxE) <= 232448, "shared memory of one CTA");
   auto kern = grouped_gemm_kernel<KIND, BN, PAIR>;
+  const size_t smem = Tr::smem_bytes(p.E);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(Tr::SMEM));
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (!PAIR) {
-    kern<<<sm_count(), Roles<KIND>::kThreads, Tr::SMEM, s>>>(m, p);
+    kern<<<sm_count(), Roles<KIND>::kThreads, smem, s>>>(m, p);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(sm_count() / 2 * 2));
   cfg.blockDim = dim3(Roles<KIND>::kThreads);
-  cfg.dynamicSmemBytes = Tr::SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -804,6 +921,7 @@ static cudaError_t launch(const Maps& m, const Params& p, cudaStream_t s) {
   return cudaLaunchKernelEx(&cfg, kern, m, p);
 }
 
+
 }  // namespace gg
 
 cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
@@ -822,6 +940,9 @@ cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   p.o0 = static_cast<bf16*>(a.h1);
   p.o1 = static_cast<bf16*>(a.h2);
   p.o2 = static_cast<bf16*>(a.a);
+  if (!make_store_map(&m1.o0, a.h1, f, rows) || !make_store_map(&m1.o1, a.h2, f, rows) ||
+      !make_store_map(&m1.o2, a.a, f, rows))
+    return cudaErrorInvalidValue;
   cudaError_t e = launch<kFwdGateUp, 256, true>(m1, p, s);
   if (e != cudaSuccess) return e;
   Maps m2{};
@@ -830,6 +951,7 @@ cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
   p.o0 = static_cast<bf16*>(a.yp);
   p.o1 = p.o2 = nullptr;
+  if (!make_store_map(&m2.o0, a.yp, d, rows)) return cudaErrorInvalidValue;
   return launch<kFwdDown, 256, true>(m2, p, s);
 }
 
@@ -855,6 +977,11 @@ cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.i1 = static_cast<const bf16*>(a.h2);
   p.o0 = static_cast<bf16*>(a.dh1);
   p.o1 = static_cast<bf16*>(a.dh2);
+  // the epilogue's h1 / h2 loads and dh1 / dh2 stores: 32 x 32 boxes
+  if (!make_store_map(&m1.a1, const_cast<void*>(a.h1), f, rows) ||
+      !make_store_map(&m1.b1, const_cast<void*>(a.h2), f, rows) ||
+      !make_store_map(&m1.o0, a.dh1, f, rows) || !make_store_map(&m1.o1, a.dh2, f, rows))
+    return cudaErrorInvalidValue;
   // 256-wide tiles even when f is not a multiple of 256 (a half-empty edge
   // tile costs less than the narrower MMA everywhere else)
   cudaError_t e = launch<kBwdDgradDown, 256, true>(m1, p, s);
@@ -867,6 +994,7 @@ cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.i0 = p.i1 = nullptr;
   p.o0 = static_cast<bf16*>(a.dxp);
   p.o1 = nullptr;
+  if (!make_store_map(&m2.o0, a.dxp, d, rows)) return cudaErrorInvalidValue;
   return launch<kBwdDgradGateUp, 256, true>(m2, p, s);
 }
 

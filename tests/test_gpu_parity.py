@@ -76,6 +76,8 @@ LAYER_CASES = [
     ("bf16_single_token", 1, 128, 4, 2, 128, "bf16", 2, False),
     ("bf16_long_k", 2048, 512, 4, 1, 256, "bf16", 1, True),
     ("bf16_f_not_256", 520, 320, 6, 2, 448, "bf16", 3, True),
+    # more experts than the deepest GEMM pipeline leaves schedule room for
+    ("bf16_many_experts", 900, 128, 160, 4, 192, "bf16", 8, True),
     ("f32_tiny", 256, 64, 4, 2, 128, "f32", 2, True),
     ("f32_odd", 100, 48, 3, 2, 20, "f32", 1, False),
 ]
