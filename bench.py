@@ -229,7 +229,9 @@ def workload_config(w):
     return {"workload": w.name, "tokens_per_gpu": w.T[0], "d_model": w.d, "experts": w.E,
             "top_k": w.k, "ffn": w.f, "ep_groups": w.ep_groups, "routing": str(w.bias),
             "l2": "inputs larger than L2 (x alone is %.0f MB; a step moves several GB); no flush"
-                  % (w.T[0] * w.d * 2 / 1e6)}
+                  % (w.T[0] * w.d * 2 / 1e6),
+            "grads": "each step writes its own fp32 parameter gradients (one microbatch per "
+                     "optimizer step)"}
 
 
 # ------------------------------------------------------------ end to end
@@ -274,7 +276,7 @@ def run_e2e(layer, x_h, dY_h, steps: int, dev, stream) -> float:
         if i + 1 < steps:
             h2d(i + 1)
         layer.forward(x_d[b], stream=stream, out=Y_d[b])
-        layer.backward(dY_d[b], stream=stream, out=dX_d[b])
+        layer.backward(dY_d[b], stream=stream, out=dX_d[b], accumulate=False)
         used[b] = torch.cuda.Event()
         used[b].record(stream)
         with torch.cuda.stream(cout):
@@ -367,9 +369,11 @@ def run_native(args, w):
     barrier = R.barrier
     max_over_ranks = R.max_over_ranks
 
+    # one microbatch per optimizer step: each step writes its own parameter
+    # gradients (no accumulation across steps)
     for _ in range(args.warmup):
         layer.forward(batch["x"])
-        layer.backward(batch["dY"])
+        layer.backward(batch["dY"], accumulate=False)
     barrier()
     errs = layer.device_errors()
     if errs:
@@ -399,7 +403,7 @@ def run_native(args, w):
         first = len(events)
         mark("step_start")
         layer.forward(batch["x"], mark=mark)
-        layer.backward(batch["dY"], mark=mark)
+        layer.backward(batch["dY"], mark=mark, accumulate=False)
         step_marks.append(first)
     end.record(stream)
     barrier()

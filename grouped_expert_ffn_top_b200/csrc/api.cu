@@ -71,6 +71,20 @@ int check_ffn(const char* fn, int dtype, int64_t rows, int E, int d, int f) {
 
 }  // namespace
 
+// accumulate = 0 on an empty batch: the requested gradient is zero. Null
+// buffers are skipped.
+static cudaError_t zero_grads(cudaStream_t stream, size_t bytes0, float* g0, size_t bytes1 = 0,
+                              float* g1 = nullptr, size_t bytes2 = 0, float* g2 = nullptr) {
+  float* g[3] = {g0, g1, g2};
+  size_t n[3] = {bytes0, bytes1, bytes2};
+  for (int i = 0; i < 3; ++i) {
+    if (!g[i]) continue;
+    cudaError_t e = cudaMemsetAsync(g[i], 0, n[i], stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 namespace moe {
 // Records the message moe_last_error() returns, for entry points defined in
 // other files of the library; returns `code`.
@@ -239,12 +253,21 @@ size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E) {
 
 int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_row,
                    const int64_t* expert_offsets, int dtype, int64_t T, int d, int E, int k,
-                   float* dWr, float* db, void* ws, size_t ws_bytes, cudaStream_t stream) {
+                   float* dWr, float* db, int accumulate, void* ws, size_t ws_bytes,
+                   cudaStream_t stream) {
   int rc = check_rows("moe_router_bwd", dtype, T, d, k);
   if (rc != MOE_OK) return rc;
   if (E < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: E=%d k=%d", E, k);
   if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd: E=%d", E);
-  if (T == 0) return MOE_OK;
+  if (accumulate != 0 && accumulate != 1)
+    return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: accumulate=%d (0 or 1)", accumulate);
+  if (T == 0) {
+    if (accumulate) return MOE_OK;
+    if (!dWr) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: null pointer");
+    return cuda_status(zero_grads(stream, sizeof(float) * static_cast<size_t>(E) * d, dWr,
+                                  sizeof(float) * E, db),
+                       "moe_router_bwd");
+  }
   if (!xp || !dlogits || !pair_of_row || !expert_offsets || !dWr || !ws)
     return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: null pointer");
   const int64_t rows = T * k;
@@ -253,8 +276,8 @@ int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_
                 moe_router_bwd_workspace_bytes(rows, d, E));
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + moe::kWsHeader);
   return launched(cuda_status(moe::launch_router_bwd(xp, dlogits, pair_of_row, expert_offsets,
-                                                      dtype, rows, d, E, k, dWr, db, partial,
-                                                      stream),
+                                                      dtype, rows, d, E, k, dWr, db, accumulate,
+                                                      partial, stream),
                               "moe_router_bwd"), 2);
 }
 
@@ -296,11 +319,18 @@ size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, in
 int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,
                         const void* h1, const void* h2, const void* a, const void* dyp, int dtype,
                         const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
-                        void* dxp, float* dWg, float* dWu, float* dWd, void* ws, size_t ws_bytes,
-                        cudaStream_t stream) {
+                        void* dxp, float* dWg, float* dWu, float* dWd, int accumulate, void* ws,
+                        size_t ws_bytes, cudaStream_t stream) {
   int rc = check_ffn("moe_grouped_ffn_bwd", dtype, rows, E, d, f);
   if (rc != MOE_OK) return rc;
-  if (rows == 0) return MOE_OK;
+  if (accumulate != 0 && accumulate != 1)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: accumulate=%d (0 or 1)", accumulate);
+  if (rows == 0) {
+    if (accumulate) return MOE_OK;
+    if (!dWg || !dWu || !dWd) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: null pointer");
+    const size_t n = sizeof(float) * static_cast<size_t>(E) * f * d;
+    return cuda_status(zero_grads(stream, n, dWg, n, dWu, n, dWd), "moe_grouped_ffn_bwd");
+  }
   if (!xp || !Wg || !Wu || !Wd || !h1 || !h2 || !a || !dyp || !expert_offsets || !dxp || !dWg ||
       !dWu || !dWd || !ws)
     return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: null pointer");
@@ -314,7 +344,7 @@ int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const vo
   const size_t h = align256(static_cast<size_t>(rows) * f * elem_bytes(dtype));
   moe::FfnBwdArgs args{xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, rows, E, d, f, dxp,
                        dWg, dWu, dWd, base + moe::kWsHeader, base + moe::kWsHeader + h,
-                       static_cast<unsigned*>(ws)};
+                       static_cast<unsigned*>(ws), accumulate};
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
                                     : moe::launch_ffn_dgrad_f32(args, stream);
   if (e == cudaSuccess) {
@@ -339,7 +369,7 @@ int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const 
     if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_dgrad: 16-byte alignment");
   if (ws_bytes < moe::kWsHeader) return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_dgrad: workspace");
   moe::FfnBwdArgs args{nullptr, Wg, Wu, Wd, h1, h2, nullptr, dyp, expert_offsets, rows, E, d, f,
-                       dxp, nullptr, nullptr, nullptr, dh1, dh2, static_cast<unsigned*>(ws)};
+                       dxp, nullptr, nullptr, nullptr, dh1, dh2, static_cast<unsigned*>(ws), 1};
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
                                     : moe::launch_ffn_dgrad_f32(args, stream);
   return launched(cuda_status(e, "moe_grouped_ffn_dgrad"), 2);
@@ -347,11 +377,18 @@ int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const 
 
 int moe_grouped_ffn_wgrad(const void* xp, const void* a, const void* dyp, const void* dh1,
                           const void* dh2, int dtype, const int64_t* expert_offsets, int64_t rows,
-                          int E, int d, int f, float* dWg, float* dWu, float* dWd, void* ws,
-                          size_t ws_bytes, cudaStream_t stream) {
+                          int E, int d, int f, float* dWg, float* dWu, float* dWd, int accumulate,
+                          void* ws, size_t ws_bytes, cudaStream_t stream) {
   int rc = check_ffn("moe_grouped_ffn_wgrad", dtype, rows, E, d, f);
   if (rc != MOE_OK) return rc;
-  if (rows == 0) return MOE_OK;
+  if (accumulate != 0 && accumulate != 1)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: accumulate=%d (0 or 1)", accumulate);
+  if (rows == 0) {
+    if (accumulate) return MOE_OK;
+    if (!dWg || !dWu || !dWd) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: null pointer");
+    const size_t n = sizeof(float) * static_cast<size_t>(E) * f * d;
+    return cuda_status(zero_grads(stream, n, dWg, n, dWu, n, dWd), "moe_grouped_ffn_wgrad");
+  }
   if (!xp || !a || !dyp || !dh1 || !dh2 || !expert_offsets || !dWg || !dWu || !dWd || !ws)
     return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: null pointer");
   const void* ptrs[] = {xp, a, dyp, dh1, dh2, dWg, dWu, dWd, ws};
@@ -360,7 +397,7 @@ int moe_grouped_ffn_wgrad(const void* xp, const void* a, const void* dyp, const 
   if (ws_bytes < moe::kWsHeader) return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_wgrad: workspace");
   moe::FfnBwdArgs args{xp, nullptr, nullptr, nullptr, nullptr, nullptr, a, dyp, expert_offsets,
                        rows, E, d, f, nullptr, dWg, dWu, dWd, const_cast<void*>(dh1),
-                       const_cast<void*>(dh2), static_cast<unsigned*>(ws)};
+                       const_cast<void*>(dh2), static_cast<unsigned*>(ws), accumulate};
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
                                     : moe::launch_ffn_wgrad_f32(args, stream);
   return launched(cuda_status(e, "moe_grouped_ffn_wgrad"), 1);

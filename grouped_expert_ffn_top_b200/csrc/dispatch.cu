@@ -404,7 +404,8 @@ __global__ void __launch_bounds__(kRbThreads) router_wgrad_partial_kernel(
 // dWr[e, c] += sum of expert e's item partials, in item order; db likewise.
 __global__ void __launch_bounds__(256) router_wgrad_reduce_kernel(
     const float* __restrict__ partial, const float* __restrict__ partial_db,
-    const int64_t* __restrict__ off, int E, int d, float* __restrict__ dWr, float* __restrict__ db) {
+    const int64_t* __restrict__ off, int E, int d, float* __restrict__ dWr, float* __restrict__ db,
+    int accumulate) {
   __shared__ int s_start[MOE_MAX_EXPERTS + 1];
   router_items_prefix(off, E, s_start);
   const int64_t n = static_cast<int64_t>(E) * d;
@@ -412,21 +413,22 @@ __global__ void __launch_bounds__(256) router_wgrad_reduce_kernel(
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int e = static_cast<int>(i / d);
     const int c = static_cast<int>(i % d);
-    if (s_start[e + 1] == s_start[e]) continue;  // no token selected e: untouched
+    // no token selected e: untouched when accumulating, zero when writing
+    if (s_start[e + 1] == s_start[e] && accumulate) continue;
     float s = 0.0f;
     for (int it = s_start[e]; it < s_start[e + 1]; ++it) s += partial[static_cast<int64_t>(it) * d + c];
-    dWr[i] += s;
+    dWr[i] = accumulate ? dWr[i] + s : s;
     if (db && c == 0) {
       float sb = 0.0f;
       for (int it = s_start[e]; it < s_start[e + 1]; ++it) sb += partial_db[it];
-      db[e] += sb;
+      db[e] = accumulate ? db[e] + sb : sb;
     }
   }
 }
 
 cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* por,
                               const int64_t* off, int dtype, int64_t rows, int d, int E, int k,
-                              float* dWr, float* db, float* partial, cudaStream_t s) {
+                              float* dWr, float* db, int accumulate, float* partial, cudaStream_t s) {
   const int items = router_bwd_max_items(rows, E);
   float* partial_db = partial + static_cast<int64_t>(items) * d;
   const int vec = dtype == MOE_BF16 ? 8 : 4;
@@ -441,7 +443,8 @@ cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* po
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(E) * d;
   const unsigned blocks = static_cast<unsigned>(((n + 255) / 256) < 148 * 8 ? (n + 255) / 256 : 148 * 8);
-  router_wgrad_reduce_kernel<<<blocks, 256, 0, s>>>(partial, partial_db, off, E, d, dWr, db);
+  router_wgrad_reduce_kernel<<<blocks, 256, 0, s>>>(partial, partial_db, off, E, d, dWr, db,
+                                                     accumulate);
   return cudaGetLastError();
 }
 

@@ -71,6 +71,7 @@ struct Params {
   float* w1;
   float* w2;
   unsigned* err;
+  int accumulate;  // wgrad: 1 adds to dW, 0 writes it (zero tiles for experts with no rows)
 };
 
 // PAIR: a cluster of two CTAs computes a 256-row tile with one
@@ -127,10 +128,12 @@ struct TileInfo {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Tiles of an expert with `cnt` rows. Writing weight gradients (accumulate
+// = 0), an expert with no rows still has its tiles: they store zeros.
 template <int KIND, int BN, bool PAIR>
-__device__ __forceinline__ int tiles_of_expert(int cnt, int d, int f) {
+__device__ __forceinline__ int tiles_of_expert(int cnt, int d, int f, int accumulate) {
   using Tr = Traits<KIND, BN, PAIR>;
-  if (cnt <= 0) return 0;
+  if (cnt <= 0 && (KIND != kWgrad || accumulate)) return 0;
   if (KIND == kWgrad)
     return 2 * ceil_div(d, Tr::TM) * ceil_div(f, BN) + ceil_div(f, Tr::TM) * ceil_div(d, BN);
   const int n_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? f : d;
@@ -312,15 +315,16 @@ __device__ __forceinline__ void red_add_f32(float* addr, float v) {
 }
 
 // Weight-gradient epilogue of one tile for this thread's accumulator row r,
-// on the columns [c0, c0 + BN / 2) of the accumulator.
+// on the columns [c0, c0 + BN / 2) of the accumulator: added to dW, or
+// written (zeros for an expert with no rows, whose tile ran no MMA).
 template <int BN>
 __device__ __forceinline__ void epilogue_wgrad(const Params& p, const TileInfo& ti, uint32_t tacc,
                                                int r, int c0) {
   // Accumulator row m, column n is element (n, m) of the [N, M] row-major
   // output, so for each column the 32 lanes of a warp cover 32 consecutive
-  // floats: one coalesced 128-byte reduction per column. red.global.add is
+  // floats: one coalesced 128-byte access per column. red.global.add is
   // fire-and-forget (the add happens at L2), and each element receives
-  // exactly one add per call, so the result is deterministic.
+  // exactly one add or store per call, so the result is deterministic.
   const int d = p.d, f = p.f;
   const int M = ti.prod == 2 ? f : d;
   const int Nn = ti.prod == 2 ? d : f;
@@ -329,13 +333,24 @@ __device__ __forceinline__ void epilogue_wgrad(const Params& p, const TileInfo& 
   float* out = (ti.prod == 0 ? p.w0 : (ti.prod == 1 ? p.w1 : p.w2)) +
                static_cast<int64_t>(ti.e) * d * f + m;
   uint32_t u[16];
+  const bool empty = ti.rows <= 0;
   for (int c = c0; c < c0 + BN / 2; c += 16) {
-    tmem_ld16(tacc + c, u);
-    tmem_ld_wait();
+    if (empty) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) u[i] = 0u;
+    } else {
+      tmem_ld16(tacc + c, u);
+      tmem_ld_wait();
+    }
     if (valid && ti.n0 + c < Nn) {
       float* q = out + static_cast<int64_t>(ti.n0 + c) * M;
+      if (p.accumulate) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) red_add_f32(q + static_cast<int64_t>(i) * M, __uint_as_float(u[i]));
+        for (int i = 0; i < 16; ++i) red_add_f32(q + static_cast<int64_t>(i) * M, __uint_as_float(u[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[static_cast<int64_t>(i) * M] = __uint_as_float(u[i]);
+      }
     }
   }
 }
@@ -627,7 +642,8 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       int v = 0;
       if (s < E) {
         const int e = s_order[s];
-        v = tiles_of_expert<KIND, BN, PAIR>(static_cast<int>(s_off[e + 1] - s_off[e]), d, f);
+        v = tiles_of_expert<KIND, BN, PAIR>(static_cast<int>(s_off[e + 1] - s_off[e]), d, f,
+                                            p.accumulate);
       }
       int inc = v;
 #pragma unroll
@@ -1010,6 +1026,7 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.w0 = a.dWg;
   p.w1 = a.dWu;
   p.w2 = a.dWd;
+  p.accumulate = a.accumulate;
   // CTA pairs: six stages of 32 KB per CTA hide more load latency than four
   // of 48 KB
   return launch<kWgrad, 256, true>(m3, p, s);

@@ -101,19 +101,20 @@ __global__ void simt_dgrad_gateup_kernel(const float* __restrict__ dh1,
   dxp[id] = s;
 }
 
-// dWg_e[j,i] += sum_r dh1[r,j] xp[r,i]; dWu_e likewise; dWd_e[i,j] += sum_r dyp[r,i] a[r,j].
-// One thread per (e, j, i); experts without rows are skipped.
+// dWg_e[j,i] (+)= sum_r dh1[r,j] xp[r,i]; dWu_e likewise; dWd_e[i,j] (+)= sum_r dyp[r,i] a[r,j].
+// One thread per (e, j, i); added when accumulating (experts without rows
+// skipped), written otherwise (zero for experts without rows).
 __global__ void simt_wgrad_kernel(const float* __restrict__ xp, const float* __restrict__ dyp,
                                   const float* __restrict__ a, const float* __restrict__ dh1,
                                   const float* __restrict__ dh2, const int64_t* __restrict__ off,
                                   int E, int d, int f, float* __restrict__ dWg,
-                                  float* __restrict__ dWu, float* __restrict__ dWd) {
+                                  float* __restrict__ dWu, float* __restrict__ dWd, int accumulate) {
   const int64_t id = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int64_t per = static_cast<int64_t>(f) * d;
   if (id >= E * per) return;
   const int e = static_cast<int>(id / per);
   const int64_t r0 = off[e], r1 = off[e + 1];
-  if (r1 == r0) return;
+  if (r1 == r0 && accumulate) return;
   const int j = static_cast<int>((id % per) / d);
   const int i = static_cast<int>(id % d);
   float sg = 0.0f, su = 0.0f, sd = 0.0f;
@@ -122,13 +123,14 @@ __global__ void simt_wgrad_kernel(const float* __restrict__ xp, const float* __r
     sg = __fmaf_rn(dh1[r * f + j], xv, sg);
     su = __fmaf_rn(dh2[r * f + j], xv, su);
   }
-  dWg[id] += sg;
-  dWu[id] += su;
+  dWg[id] = accumulate ? dWg[id] + sg : sg;
+  dWu[id] = accumulate ? dWu[id] + su : su;
   // dWd_e is [d, f]; reuse the thread for element (i', j') = (j*d+i) / f, % f
   const int64_t q = id % per;
   const int di = static_cast<int>(q / f), fj = static_cast<int>(q % f);
   for (int64_t r = r0; r < r1; ++r) sd = __fmaf_rn(dyp[r * d + di], a[r * f + fj], sd);
-  dWd[static_cast<int64_t>(e) * per + q] += sd;
+  float* od = dWd + static_cast<int64_t>(e) * per + q;
+  *od = accumulate ? *od + sd : sd;
 }
 
 static unsigned blocks_for(int64_t n) { return static_cast<unsigned>((n + 255) / 256); }
@@ -167,7 +169,8 @@ cudaError_t launch_ffn_wgrad_f32(const FfnBwdArgs& x, cudaStream_t s) {
   const float* dh2 = static_cast<const float*>(x.dh2);
   simt_wgrad_kernel<<<blocks_for(static_cast<int64_t>(x.E) * x.f * x.d), 256, 0, s>>>(
       static_cast<const float*>(x.xp), static_cast<const float*>(x.dyp),
-      static_cast<const float*>(x.a), dh1, dh2, x.offsets, x.E, x.d, x.f, x.dWg, x.dWu, x.dWd);
+      static_cast<const float*>(x.a), dh1, dh2, x.offsets, x.E, x.d, x.f, x.dWg, x.dWu, x.dWd,
+      x.accumulate);
   return cudaGetLastError();
 }
 

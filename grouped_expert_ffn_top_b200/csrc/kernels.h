@@ -41,7 +41,7 @@ cudaError_t launch_permute_bwd(const void* dxp, const int32_t* row_of_pair, cons
 int router_bwd_max_items(int64_t rows, int E);
 cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* pair_of_row,
                               const int64_t* offsets, int dtype, int64_t rows, int d, int E, int k,
-                              float* dWr, float* db, float* partial, cudaStream_t s);
+                              float* dWr, float* db, int accumulate, float* partial, cudaStream_t s);
 
 // grouped expert FFN (grouped_gemm_sm100.cu, grouped_simt.cu)
 struct FfnFwdArgs {
@@ -61,6 +61,7 @@ struct FfnBwdArgs {
   float *dWg, *dWu, *dWd;
   void *dh1, *dh2;  // [rows, f]: written by dgrad, read by wgrad
   unsigned* err;
+  int accumulate;   // wgrad: 1 adds to dW, 0 writes dW (zero for experts with no rows)
 };
 
 cudaError_t launch_selftest_wait_timeout(unsigned* err, long long limit, cudaStream_t s);

@@ -8,7 +8,9 @@ Backward: moe_unpermute_combine_bwd -> moe_route_bwd -> moe_grouped_ffn_dgrad
 
 The object owns device buffers sized for `max_tokens`, so a step allocates
 nothing; microbatches of any size up to that (0 included) reuse them. Weight
-gradients accumulate in fp32 across microbatches until zero_grad().
+gradients accumulate in fp32 across microbatches until zero_grad(); a
+backward with accumulate=False writes them instead (the first microbatch of a
+step: the old values are neither read nor needed).
 """
 from __future__ import annotations
 
@@ -128,9 +130,11 @@ class MoELayer:
         mark("unpermute_combine")
         return Y
 
-    def backward(self, dY: torch.Tensor, stream=None, mark=None, out=None) -> torch.Tensor:
+    def backward(self, dY: torch.Tensor, stream=None, mark=None, out=None,
+                 accumulate: bool = True) -> torch.Tensor:
         """dX for upstream gradient dY of the last forward (written to `out`
-        if given); dW += (fp32)."""
+        if given); dW += the batch's gradient (fp32), or dW = it if not
+        `accumulate`."""
         mark = mark or _no_mark
         T = self.T
         v, r = self.v, self.r
@@ -143,14 +147,14 @@ class MoELayer:
                                 v["dh1"], v["dh2"], v["dxp"], self.ws["ffn_bwd"], stream)
         mark("grouped_ffn_dgrad")
         N.moe_grouped_ffn_wgrad(v["xp"], v["a"], v["dyp"], v["dh1"], v["dh2"], r["offsets"], g["dWg"],
-                                g["dWu"], g["dWd"], self.ws["ffn_bwd"], stream)
+                                g["dWu"], g["dWd"], self.ws["ffn_bwd"], stream, accumulate=accumulate)
         mark("grouped_ffn_wgrad")
         dX = v["dX"] if out is None else out
         N.moe_permute_bwd(v["dxp"], r["row_of_pair"], v["dlogits"], self.Wr, r["topk_idx"], T, self.k,
                           dX, stream)
         mark("permute_bwd")
         N.moe_router_bwd(v["xp"], v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"], g["db"],
-                         self.ws["router_bwd"], stream)
+                         self.ws["router_bwd"], stream, accumulate=accumulate)
         mark("router_bwd")
         return dX
 

@@ -60,12 +60,12 @@ _SIGNATURES = {
     "moe_unpermute_combine_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _p, _p, _p], _i),
     "moe_route_bwd": ([_p, _p, _p, _i64, _i, _i, _p, _p], _i),
     "moe_grouped_ffn_bwd_workspace_bytes": ([_i64, _i, _i, _i, _i], _sz),
-    "moe_grouped_ffn_bwd": ([_p] * 8 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_grouped_ffn_bwd": ([_p] * 8 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _i, _p, _sz, _p], _i),
     "moe_grouped_ffn_dgrad": ([_p] * 6 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
-    "moe_grouped_ffn_wgrad": ([_p] * 5 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_grouped_ffn_wgrad": ([_p] * 5 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _i, _p, _sz, _p], _i),
     "moe_permute_bwd": ([_p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p], _i),
     "moe_router_bwd_workspace_bytes": ([_i64, _i, _i], _sz),
-    "moe_router_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p, _p, _sz, _p], _i),
+    "moe_router_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p, _i, _p, _sz, _p], _i),
 }
 
 
@@ -249,7 +249,7 @@ def moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype) -> int:
 
 
 def moe_grouped_ffn_bwd(xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu, dWd,
-                        dxp=None, ws=None, stream=None):
+                        dxp=None, ws=None, stream=None, accumulate: bool = True):
     _contig(xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu, dWd)
     rows, d = xp.shape
     E, f, _ = Wg.shape
@@ -260,8 +260,8 @@ def moe_grouped_ffn_bwd(xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu
         ws = _ws(moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dt), xp.device)
     _check(lib().moe_grouped_ffn_bwd(_ptr(xp), _ptr(Wg), _ptr(Wu), _ptr(Wd), _ptr(h1), _ptr(h2),
                                      _ptr(a), _ptr(dyp), dt, _ptr(expert_offsets), rows, E, d, f,
-                                     _ptr(dxp), _ptr(dWg), _ptr(dWu), _ptr(dWd), _ptr(ws), ws.numel(),
-                                     _stream(stream)), "moe_grouped_ffn_bwd")
+                                     _ptr(dxp), _ptr(dWg), _ptr(dWu), _ptr(dWd), int(accumulate), _ptr(ws),
+                                     ws.numel(), _stream(stream)), "moe_grouped_ffn_bwd")
     return dxp
 
 
@@ -276,13 +276,15 @@ def moe_grouped_ffn_dgrad(Wg, Wu, Wd, h1, h2, dyp, expert_offsets, dh1, dh2, dxp
     return dxp
 
 
-def moe_grouped_ffn_wgrad(xp, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd, ws, stream=None):
+def moe_grouped_ffn_wgrad(xp, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd, ws, stream=None,
+                          accumulate: bool = True):
     _contig(xp, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd)
     rows, d = xp.shape
     E, f, _ = dWg.shape
     _check(lib().moe_grouped_ffn_wgrad(_ptr(xp), _ptr(a), _ptr(dyp), _ptr(dh1), _ptr(dh2), _dt(xp),
                                        _ptr(expert_offsets), rows, E, d, f, _ptr(dWg), _ptr(dWu),
-                                       _ptr(dWd), _ptr(ws), ws.numel(), _stream(stream)),
+                                       _ptr(dWd), int(accumulate), _ptr(ws), ws.numel(),
+                                       _stream(stream)),
            "moe_grouped_ffn_wgrad")
 
 
@@ -301,12 +303,13 @@ def moe_router_bwd_workspace_bytes(rows, d, E) -> int:
     return lib().moe_router_bwd_workspace_bytes(rows, d, E)
 
 
-def moe_router_bwd(xp, dlogits, pair_of_row, expert_offsets, k: int, dWr, db, ws=None, stream=None):
+def moe_router_bwd(xp, dlogits, pair_of_row, expert_offsets, k: int, dWr, db, ws=None, stream=None,
+                   accumulate: bool = True):
     _contig(xp, dlogits, pair_of_row, expert_offsets, dWr, db)
     rows, d = xp.shape
     T, E = dlogits.shape
     if ws is None:
         ws = _ws(moe_router_bwd_workspace_bytes(rows, d, E), xp.device)
     _check(lib().moe_router_bwd(_ptr(xp), _ptr(dlogits), _ptr(pair_of_row), _ptr(expert_offsets),
-                                _dt(xp), T, d, E, k, _ptr(dWr), _ptr(db), _ptr(ws), ws.numel(),
-                                _stream(stream)), "moe_router_bwd")
+                                _dt(xp), T, d, E, k, _ptr(dWr), _ptr(db), int(accumulate), _ptr(ws),
+                                ws.numel(), _stream(stream)), "moe_router_bwd")

@@ -40,9 +40,13 @@
  *     synchronises.
  *   - T = 0 (an empty microbatch) is valid everywhere: the call returns
  *     MOE_OK, launches nothing and leaves every output and accumulator as it
- *     was.
- *   - Gradients of parameters accumulate (+=) into fp32 buffers the caller
- *     zeroes before the first microbatch; activation gradients overwrite.
+ *     was (except that a parameter gradient requested with accumulate = 0 is
+ *     set to zero, the gradient of an empty batch).
+ *   - Gradients of parameters go to fp32 buffers: with accumulate = 1 they
+ *     are added (+=, gradient accumulation over microbatches), with
+ *     accumulate = 0 they are written (=, the first microbatch of a step;
+ *     the buffer's old contents are not read). Activation gradients
+ *     overwrite.
  *   - Return value: MOE_OK, or a negative MOE_ERR_* code with a message
  *     available from moe_last_error() (thread-local). Arguments are checked
  *     before anything is launched; a rejected call changes nothing.
@@ -246,16 +250,18 @@ MOE_API size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, i
 /* Grouped SwiGLU expert FFN, backward. Per expert e over its rows:
  *   da  = dyp Wd_e;  dh1 = da * h2 * silu'(h1);  dh2 = da * silu(h1)
  *   dxp = dh1 Wg_e + dh2 Wu_e                           (overwritten)
- *   dWg_e += dh1^T xp;  dWu_e += dh2^T xp;  dWd_e += dyp^T a   (fp32, +=)
- * with silu'(u) = s (1 + u (1 - s)), s = sigmoid(u). An expert with no rows
- * leaves its gradients untouched.
+ *   dWg_e += dh1^T xp;  dWu_e += dh2^T xp;  dWd_e += dyp^T a   (fp32)
+ * with silu'(u) = s (1 + u (1 - s)), s = sigmoid(u). accumulate = 1: the
+ * products are added to dW, and an expert with no rows leaves its gradients
+ * untouched; accumulate = 0: dW is overwritten with the products (zero for
+ * an expert with no rows) and never read.
  *   xp, dyp [rows, d]; h1, h2, a [rows, f]; Wg, Wu [E, f, d]; Wd [E, d, f]
- *   dxp [rows, d] dtype output; dWg, dWu [E, f, d], dWd [E, d, f] fp32 (+=).
+ *   dxp [rows, d] dtype output; dWg, dWu [E, f, d], dWd [E, d, f] fp32.
  * Errors: as moe_grouped_ffn_fwd. */
 MOE_API int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,
                         const void* h1, const void* h2, const void* a, const void* dyp,
                         int dtype, const int64_t* expert_offsets, int64_t rows, int E, int d,
-                        int f, void* dxp, float* dWg, float* dWu, float* dWd,
+                        int f, void* dxp, float* dWg, float* dWu, float* dWd, int accumulate,
                         void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* The two halves of moe_grouped_ffn_bwd, for callers that keep dh1 / dh2
@@ -264,8 +270,9 @@ MOE_API int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, 
  * moe_grouped_ffn_dgrad: data gradients
  *   dh1, dh2 [rows, f] dtype outputs (the SwiGLU backward of da = dyp Wd_e)
  *   dxp [rows, d] dtype output (= dh1 Wg_e + dh2 Wu_e)
- * moe_grouped_ffn_wgrad: weight gradients, accumulated in fp32
- *   dWg_e += dh1^T xp; dWu_e += dh2^T xp; dWd_e += dyp^T a
+ * moe_grouped_ffn_wgrad: weight gradients in fp32, added or written as the
+ * accumulate flag says (as moe_grouped_ffn_bwd)
+ *   dWg_e (+)= dh1^T xp; dWu_e (+)= dh2^T xp; dWd_e (+)= dyp^T a
  * ws needs moe_grouped_ffn_fwd_workspace_bytes() bytes (its error word). */
 MOE_API int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const void* h1,
                                   const void* h2, const void* dyp, int dtype,
@@ -275,7 +282,8 @@ MOE_API int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd
 MOE_API int moe_grouped_ffn_wgrad(const void* xp, const void* a, const void* dyp, const void* dh1,
                                   const void* dh2, int dtype, const int64_t* expert_offsets,
                                   int64_t rows, int E, int d, int f, float* dWg, float* dWu,
-                                  float* dWd, void* ws, size_t ws_bytes, cudaStream_t stream);
+                                  float* dWd, int accumulate, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream);
 
 /* Permute backward, with the router's input gradient folded in:
  *   dX[t, :] = sum_{j<k} dxp[row_of_pair[t*k+j], :]
@@ -294,8 +302,9 @@ MOE_API int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const f
 /* Workspace of moe_router_bwd, in bytes (rows = T*k). */
 MOE_API size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E);
 
-/* Router weight gradients (accumulated, fp32, deterministic order):
- *   dWr[e, :] += sum_t dlogits[t, e] x[t, :];   db[e] += sum_t dlogits[t, e]
+/* Router weight gradients (fp32, deterministic order; added with
+ * accumulate = 1, written with accumulate = 0):
+ *   dWr[e, :] (+)= sum_t dlogits[t, e] x[t, :];   db[e] (+)= sum_t dlogits[t, e]
  * (router backward of z = x Wr^T + b). The sums run over the dispatch rows
  * instead of all tokens: expert e's rows [expert_offsets[e],
  * expert_offsets[e+1]) hold exactly the tokens that selected e, and xp holds
@@ -306,11 +315,12 @@ MOE_API size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E);
  * T x E x d product.
  *   xp [T*k, d] dtype (moe_permute's output); dlogits [T, E] fp32;
  *   pair_of_row [T*k], expert_offsets [E+1] (moe_route's outputs);
- *   dWr [E, d] fp32 (+=); db [E] fp32 (+=, may be NULL). */
+ *   dWr [E, d] fp32; db [E] fp32 (may be NULL). An expert no token selected
+ * keeps its rows (accumulate = 1) or gets zeros (accumulate = 0). */
 MOE_API int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_row,
                            const int64_t* expert_offsets, int dtype, int64_t T, int d, int E,
-                           int k, float* dWr, float* db, void* ws, size_t ws_bytes,
-                           cudaStream_t stream);
+                           int k, float* dWr, float* db, int accumulate, void* ws,
+                           size_t ws_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -100,7 +100,22 @@ def test_row_pass_argument_errors(L):
     assert L.moe_permute_bwd(null, null, null, null, null, N.MOE_BF16, 4, 128, 2, 3, null, null) == \
         N.MOE_ERR_INVALID_ARG  # k > E
     assert L.moe_route_bwd(null, null, null, 4, 8, 9, null, null) == N.MOE_ERR_INVALID_ARG
-    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 0, 128, 8, 2, null, null, null, 0,
+    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 0, 128, 8, 2, null, null, 1, null, 0,
                             null) == N.MOE_OK
-    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 4, 128, 8, 9, null, null, null, 0,
+    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 4, 128, 8, 9, null, null, 1, null, 0,
                             null) == N.MOE_ERR_INVALID_ARG
+    # accumulate must be 0 or 1; writing the gradient of an empty batch needs the buffer
+    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 0, 128, 8, 2, null, null, 2, null, 0,
+                            null) == N.MOE_ERR_INVALID_ARG
+    assert L.moe_router_bwd(null, null, null, null, N.MOE_BF16, 0, 128, 8, 2, null, null, 0, null, 0,
+                            null) == N.MOE_ERR_INVALID_ARG
+
+
+def test_wgrad_accumulate_flag_errors(L):
+    args = [null] * 5 + [N.MOE_BF16, null, 0, 4, 128, 128, null, null, null]
+    assert L.moe_grouped_ffn_wgrad(*args, 1, null, 0, null) == N.MOE_OK  # empty batch, adding
+    assert L.moe_grouped_ffn_wgrad(*args, 2, null, 0, null) == N.MOE_ERR_INVALID_ARG
+    assert L.moe_grouped_ffn_wgrad(*args, 0, null, 0, null) == N.MOE_ERR_INVALID_ARG  # null dW
+    bargs = [null] * 8 + [N.MOE_BF16, null, 0, 4, 128, 128, null, null, null, null]
+    assert L.moe_grouped_ffn_bwd(*bargs, 1, null, 0, null) == N.MOE_OK
+    assert L.moe_grouped_ffn_bwd(*bargs, 0, null, 0, null) == N.MOE_ERR_INVALID_ARG

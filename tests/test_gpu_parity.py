@@ -241,6 +241,39 @@ def test_long_ragged_weight_gradient_is_exact_and_reproducible():
         assert torch.equal(layer.grads[n], first[n]), n
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_without_accumulate_writes_the_gradients(dtype):
+    """accumulate=False: parameter gradients are written, whatever the
+    buffers held (an expert no token selected gets zeros), and an empty
+    microbatch writes zeros."""
+    T, d, E, k, f = (700, 256, 8, 2, 384) if dtype == "bf16" else (200, 64, 4, 2, 128)
+    w, p, bt = _layer_case(T, d, E, k, f, dtype, 2, True, seed=9)
+    tol = TOL[w.torch_dtype()]
+    layer = MoELayer(p, k, 2, max_tokens=T)
+    for n, g in layer.grads.items():
+        g.fill_(1.0e3)
+    layer.forward(bt["x"])
+    layer.backward(bt["dY"], accumulate=False)
+    torch.cuda.synchronize()
+    assert layer.device_errors() == 0
+    P = _np_params(p)
+    x64 = to_np(bt["x"]).astype(np.float64)
+    fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k, 2)
+    bw = oracle.layer_backward(fw, x64, to_np(bt["dY"]).astype(np.float64), P["Wr"], P["Wg"], P["Wu"],
+                               P["Wd"], k)
+    for n in ("dWg", "dWu", "dWd", "dWr", "db"):
+        assert_close(n, layer.grads[n], bw[n], tol)
+    for n in ("dWg", "dWu", "dWd", "dWr"):
+        assert not layer.grads[n][E - 1].any(), f"{n} of the starved expert must be written as zero"
+    # an empty microbatch without accumulation: the gradient of nothing is zero
+    x0 = torch.empty((0, d), dtype=w.torch_dtype(), device=DEV)
+    layer.forward(x0)
+    layer.backward(x0, accumulate=False)
+    torch.cuda.synchronize()
+    for n, g in layer.grads.items():
+        assert not g.any(), n
+
+
 # ----------------------------------------------------- failure detection
 
 def test_bounded_wait_times_out_and_leaves_the_context_usable():
