@@ -721,20 +721,44 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, s_abort, kWaitLimit)) break;
       tc_fence_after();
       const uint32_t dtm = tmem_base + acc * BN;
-      for (int kb = 0; kb < nk; ++kb) {
+      // Full 64-deep K blocks: four MMAs each as straight-line code (a loop
+      // with a run-time bound, or a branch, between them leaves the tensor
+      // pipe idle between instructions).
+      const int nfull = KIND == kWgrad ? ti.rows / BK : nk;
+      for (int kb = 0; kb < nfull; ++kb) {
         if (!wait_bounded(&full[stage], phase, s_abort, kWaitLimit)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        int ksteps = BK / 16;
-        if (KIND == kWgrad && (kb + 1) * BK > ti.rows) {
-          // ragged-K tail: rows past the expert's end belong to the next
-          // expert (or lie past the tensor). Only the 16-row MMA steps that
-          // hold valid rows run, and the invalid rows inside the last of them
-          // are zeroed in both operands first.
+        if (lane == 0) {
+          const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, (kb | kk) != 0 ? 1u : 0u);
+          // the stage is free in both CTAs once these MMAs have read it
+          if (PAIR) mma_commit_pair_multicast(&empty[stage], 0x3);
+          else mma_commit(&empty[stage]);
+        }
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (KIND == kWgrad && ok && nfull < nk) {
+        // ragged-K tail block: rows past the expert's end belong to the next
+        // expert (or lie past the tensor). Only the 16-row MMA steps that
+        // hold valid rows run, and the invalid rows inside the last of them
+        // are zeroed in both operands first.
+        const int kb = nfull;
+        if (!wait_bounded(&full[stage], phase, s_abort, kWaitLimit)) {
+          ok = false;
+        } else {
+          tc_fence_after();
           const int valid = ti.rows - kb * BK;
-          ksteps = (valid + 15) / 16;
+          const int ksteps = (valid + 15) / 16;
           const int zrows = ksteps * 16 - valid;
           if (zrows > 0) {
             // each 64-column box holds one 128-byte row per K row, so the rows
@@ -756,29 +780,19 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
             else fence_proxy_async_smem();
           }
           __syncwarp();
-        }
-        if (lane == 0) {
-          const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
-          const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
-          // A full block issues its four MMAs as straight-line code: a loop
-          // with a run-time bound between them leaves the tensor pipe idle
-          // between instructions. Only a ragged wgrad tail takes the loop.
-          if (ksteps == BK / 16) {
-#pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, (kb | kk) != 0 ? 1u : 0u);
-          } else {
+          if (lane == 0) {
+            const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
+            const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
             for (int kk = 0; kk < ksteps; ++kk)
               issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, (kb | kk) != 0 ? 1u : 0u);
+            if (PAIR) mma_commit_pair_multicast(&empty[stage], 0x3);
+            else mma_commit(&empty[stage]);
           }
-          // the stage is free in both CTAs once these MMAs have read it
-          if (PAIR) mma_commit_pair_multicast(&empty[stage], 0x3);
-          else mma_commit(&empty[stage]);
-        }
-        __syncwarp();
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
+          __syncwarp();
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
       if (!ok) break;
