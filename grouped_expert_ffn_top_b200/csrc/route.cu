@@ -12,47 +12,64 @@ namespace moe {
 // ------------------------------------------------------------ router logits
 //
 // z[t,e] = fma-chain over i = 0..d-1 of x[t,i] * Wr[e,i], then + b[e], in fp32.
-// Block tile: 64 tokens x TE experts, 64 threads; thread tile: 8 tokens x
-// TE/8 experts. Operands are staged as fp32 in shared memory, i-major, in
-// chunks of 64 i: each thread loads its token row's chunk with 16-byte vector
-// loads one chunk ahead (register double buffer) and writes it transposed.
-// The i loop is sequential for every output, which is what makes the result
-// bit-identical to the fixed-order definition.
+// Block tile: 64 tokens x TE experts, NT threads in 8 token groups of 8
+// tokens and NT / 8 expert groups; thread tile: 8 tokens x TE / (NT / 8)
+// experts. Operands are staged as fp32 in shared memory, i-major, in chunks
+// of 64 i, loaded with 16-byte vector loads one chunk ahead (register double
+// buffer) and written transposed; each 32-float half of a staged row is
+// followed by 16 bytes of padding, so that the 16-byte operand loads of the
+// token and expert groups fall in distinct banks. Within a chunk the next
+// step's operands load into a second register set while the current step's
+// FMAs issue. The i loop is
+// sequential for every output, which is what makes the result bit-identical
+// to the fixed-order definition.
 
 constexpr int kLogitTokens = 64;
 constexpr int kLogitChunk = 64;
 
-template <typename T, int TE>
-__global__ void __launch_bounds__(64) router_logits_kernel(const T* __restrict__ x,
+// padded column of element c of a staged row: 4 floats after every 32
+__device__ __forceinline__ int logit_pad(int c) { return c + ((c >> 5) << 2); }
+
+template <typename T, int TE, int NT>
+__global__ void __launch_bounds__(NT) router_logits_kernel(const T* __restrict__ x,
                                                            const T* __restrict__ Wr,
                                                            const float* __restrict__ b,
                                                            int64_t Ttok, int d, int E,
                                                            float* __restrict__ z) {
-  constexpr int VE = Vec16<T>::N;              // elements per 16-byte vector
-  constexpr int VPR = kLogitChunk / VE;        // vectors per row chunk
-  constexpr int WPT = TE * VPR / 64;           // Wr vectors per thread
-  constexpr int RE = TE / 8;                   // experts per thread
-  static_assert(TE * VPR % 64 == 0, "Wr staging");
-  __shared__ __align__(16) float xs[kLogitChunk][kLogitTokens];
-  __shared__ __align__(16) float ws[kLogitChunk][TE];
+  constexpr int VE = Vec16<T>::N;                  // elements per 16-byte vector
+  constexpr int VPR = kLogitChunk / VE;            // vectors per row chunk
+  constexpr int XPT = kLogitTokens * VPR / NT;     // x vectors per thread
+  constexpr int WPT = TE * VPR / NT;               // Wr vectors per thread
+  constexpr int EG = NT / 8;                       // expert groups
+  constexpr int RE = TE / EG;                      // experts per thread
+  constexpr int XROW = kLogitTokens + kLogitTokens / 32 * 4;
+  constexpr int WROW = TE + (TE + 31) / 32 * 4;
+  static_assert(XPT >= 1 && kLogitTokens * VPR % NT == 0, "x staging");
+  static_assert(WPT >= 1 && TE * VPR % NT == 0, "Wr staging");
+  static_assert(RE >= 1 && TE % EG == 0, "thread tile");
+  __shared__ __align__(16) float xs[kLogitChunk][XROW];
+  __shared__ __align__(16) float ws[kLogitChunk][WROW];
   const int tid = threadIdx.x;
-  const int tx = tid % 8;  // expert group
-  const int ty = tid / 8;  // token group
+  const int tx = tid % EG;  // expert group
+  const int ty = tid / EG;  // token group
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kLogitTokens;
   const int e0 = blockIdx.y * TE;
-  const int64_t my_t = t0 + tid;
+  // x staging: thread tid loads token tid % 64, vectors (tid / 64) * XPT ..
+  const int xt = tid % kLogitTokens;
+  const int xv0 = (tid / kLogitTokens) * XPT;
+  const int64_t my_t = t0 + xt;
 
-  Vec16<T> xr[VPR], wr[WPT];
+  Vec16<T> xr[XPT], wr[WPT];
   auto load_stage = [&](int i0) {
 #pragma unroll
-    for (int v = 0; v < VPR; ++v) {
-      const int i = i0 + v * VE;
+    for (int v = 0; v < XPT; ++v) {
+      const int i = i0 + (xv0 + v) * VE;
       if (my_t < Ttok && i < d) xr[v] = ld16_stream(x + my_t * d + i);
       else xr[v].raw = make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int j = 0; j < WPT; ++j) {
-      const int vid = tid + 64 * j;
+      const int vid = tid + NT * j;
       const int ee = vid % TE, v = vid / TE;
       const int e = e0 + ee, i = i0 + v * VE;
       if (e < E && i < d) wr[j] = ld16(Wr + static_cast<int64_t>(e) * d + i);
@@ -69,33 +86,53 @@ __global__ void __launch_bounds__(64) router_logits_kernel(const T* __restrict__
   load_stage(0);
   for (int i0 = 0; i0 < d; i0 += kLogitChunk) {
 #pragma unroll
-    for (int v = 0; v < VPR; ++v)
+    for (int v = 0; v < XPT; ++v)
 #pragma unroll
-      for (int q = 0; q < VE; ++q) xs[v * VE + q][tid] = xr[v].get(q);
+      for (int q = 0; q < VE; ++q) xs[(xv0 + v) * VE + q][logit_pad(xt)] = xr[v].get(q);
 #pragma unroll
     for (int j = 0; j < WPT; ++j) {
-      const int vid = tid + 64 * j;
+      const int vid = tid + NT * j;
       const int ee = vid % TE, v = vid / TE;
 #pragma unroll
-      for (int q = 0; q < VE; ++q) ws[v * VE + q][ee] = wr[j].get(q);
+      for (int q = 0; q < VE; ++q) ws[v * VE + q][logit_pad(ee)] = wr[j].get(q);
     }
     __syncthreads();
     if (i0 + kLogitChunk < d) load_stage(i0 + kLogitChunk);
     const int iend = min(kLogitChunk, d - i0);
-#pragma unroll 4
-    for (int ii = 0; ii < iend; ++ii) {
-      float xv[8], wv[RE];
-      const float4 xa = *reinterpret_cast<const float4*>(&xs[ii][ty * 8]);
-      const float4 xb = *reinterpret_cast<const float4*>(&xs[ii][ty * 8 + 4]);
-      xv[0] = xa.x; xv[1] = xa.y; xv[2] = xa.z; xv[3] = xa.w;
-      xv[4] = xb.x; xv[5] = xb.y; xv[6] = xb.z; xv[7] = xb.w;
+    // two register sets alternate: step ii + 1 loads into one while step
+    // ii's FMAs read the other
+    float xa[8], wa[RE], xb[8], wb[RE];
+    auto load_step = [&](int ii, float (&xv)[8], float (&wv)[RE]) {
+      const float4 x0 = *reinterpret_cast<const float4*>(&xs[ii][logit_pad(ty * 8)]);
+      const float4 x1 = *reinterpret_cast<const float4*>(&xs[ii][logit_pad(ty * 8) + 4]);
+      xv[0] = x0.x; xv[1] = x0.y; xv[2] = x0.z; xv[3] = x0.w;
+      xv[4] = x1.x; xv[5] = x1.y; xv[6] = x1.z; xv[7] = x1.w;
+      if constexpr (RE % 4 == 0) {
 #pragma unroll
-      for (int c = 0; c < RE; ++c) wv[c] = ws[ii][tx * RE + c];
+        for (int c = 0; c < RE; c += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(&ws[ii][logit_pad(tx * RE + c)]);
+          wv[c] = w4.x; wv[c + 1] = w4.y; wv[c + 2] = w4.z; wv[c + 3] = w4.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < RE; ++c) wv[c] = ws[ii][logit_pad(tx * RE + c)];
+      }
+    };
+    auto fma_step = [&](const float (&xv)[8], const float (&wv)[RE]) {
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int c = 0; c < RE; ++c) acc[a][c] = __fmaf_rn(xv[a], wv[c], acc[a][c]);
+    };
+    load_step(0, xa, wa);
+    int ii = 0;
+    for (; ii + 1 < iend; ii += 2) {
+      load_step(ii + 1, xb, wb);
+      fma_step(xa, wa);
+      if (ii + 2 < iend) load_step(ii + 2, xa, wa);
+      fma_step(xb, wb);
     }
+    if (ii < iend) fma_step(xa, wa);  // odd chunk length (fp32 rows)
     __syncthreads();
   }
 #pragma unroll
@@ -115,13 +152,14 @@ static cudaError_t launch_router_logits_t(const T* x, const T* Wr, const float* 
                                           int d, int E, float* z, cudaStream_t s) {
   const unsigned gx = static_cast<unsigned>((Ttok + kLogitTokens - 1) / kLogitTokens);
   if (E <= 8) {
-    router_logits_kernel<T, 8><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 8, 64><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 16) {
-    router_logits_kernel<T, 16><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 16, 128><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 32) {
-    router_logits_kernel<T, 32><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 32, 128><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else {
-    router_logits_kernel<T, 64><<<dim3(gx, (E + 63) / 64), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    router_logits_kernel<T, 64, 128><<<dim3(gx, (E + 63) / 64), 128, 0, s>>>(x, Wr, b, Ttok, d,
+                                                                             E, z);
   }
   return cudaGetLastError();
 }
