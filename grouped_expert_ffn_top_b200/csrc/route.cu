@@ -194,8 +194,8 @@ __device__ __forceinline__ bool ranks_before(const Cand& a, const Cand& b) {
   return a.idx < b.idx;
 }
 
-template <int S>  // S = ceil(E / 32) logits per lane
-__global__ void __launch_bounds__(kRouteThreads) topk_softmax_kernel(
+template <int S, int NT>  // S = ceil(E / 32) logits per lane, NT threads per block
+__global__ void __launch_bounds__(NT) topk_softmax_kernel(
     const float* __restrict__ z, int64_t Ttok, int E, int k, int32_t* __restrict__ topk_idx,
     float* __restrict__ topk_w, int32_t* __restrict__ block_counts, unsigned* err) {
   extern __shared__ int s_hist[];  // [E]
@@ -205,7 +205,17 @@ __global__ void __launch_bounds__(kRouteThreads) topk_softmax_kernel(
   __syncthreads();
 
   const int64_t tok_base = static_cast<int64_t>(blockIdx.x) * kRouteTokensPerBlock;
-  constexpr int kTokPerWarp = kRouteTokensPerBlock / (kRouteThreads / 32);
+  constexpr int kTokPerWarp = kRouteTokensPerBlock / (NT / 32);
+  // the next token's logits load while this one is ranked
+  float vn[S];
+  auto load_token = [&](int64_t t) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+      const int e = lane + 32 * s;
+      vn[s] = (t < Ttok && e < E) ? z[t * E + e] : 0.0f;
+    }
+  };
+  load_token(tok_base + warp * kTokPerWarp);
   for (int q = 0; q < kTokPerWarp; ++q) {
     const int64_t t = tok_base + warp * kTokPerWarp + q;
     if (t >= Ttok) break;
@@ -213,10 +223,10 @@ __global__ void __launch_bounds__(kRouteThreads) topk_softmax_kernel(
     bool taken[S];
 #pragma unroll
     for (int s = 0; s < S; ++s) {
-      const int e = lane + 32 * s;
-      v[s] = e < E ? z[t * E + e] : 0.0f;
-      taken[s] = e >= E;
+      v[s] = vn[s];
+      taken[s] = lane + 32 * s >= E;
     }
+    if (q + 1 < kTokPerWarp) load_token(t + 1);
     float my_val = 0.0f;  // lane j keeps the j-th selected logit
     int my_idx = 0;
     for (int j = 0; j < k; ++j) {
@@ -391,6 +401,20 @@ __global__ void __launch_bounds__(kRouteThreads) route_scatter_kernel(
   }
 }
 
+// 1024 threads (8 tokens per warp) while a lane's logits fit in a few
+// registers (E <= 128), else 256.
+template <int SV>
+static void launch_topk(int nb, size_t smem, cudaStream_t s, const float* z, int64_t T, int E,
+                        int k, int32_t* topk_idx, float* topk_w, int32_t* block_counts,
+                        unsigned* err) {
+  if constexpr (SV <= 4)
+    topk_softmax_kernel<SV, 1024><<<nb, 1024, smem, s>>>(z, T, E, k, topk_idx, topk_w,
+                                                          block_counts, err);
+  else
+    topk_softmax_kernel<SV, kRouteThreads><<<nb, kRouteThreads, smem, s>>>(z, T, E, k, topk_idx,
+                                                                           topk_w, block_counts, err);
+}
+
 cudaError_t launch_route(const float* z, int64_t T, int E, int k, int G, int32_t* topk_idx,
                          float* topk_w, int32_t* counts, int64_t* offsets, int32_t* group_counts,
                          int64_t* group_offsets, int32_t* row_of_pair, int32_t* pair_of_row,
@@ -399,16 +423,12 @@ cudaError_t launch_route(const float* z, int64_t T, int E, int k, int G, int32_t
   const int nb = static_cast<int>((T + kRouteTokensPerBlock - 1) / kRouteTokensPerBlock);
   const size_t hist_smem = sizeof(int) * E;
   const int S = (E + 31) / 32;
-#define MOE_TOPK_CASE(SV)                                                                  \
-  topk_softmax_kernel<SV><<<nb, kRouteThreads, hist_smem, s>>>(z, T, E, k, topk_idx, topk_w, \
-                                                               block_counts, err)
-  if (S <= 1) MOE_TOPK_CASE(1);
-  else if (S <= 2) MOE_TOPK_CASE(2);
-  else if (S <= 4) MOE_TOPK_CASE(4);
-  else if (S <= 8) MOE_TOPK_CASE(8);
-  else if (S <= 16) MOE_TOPK_CASE(16);
-  else MOE_TOPK_CASE(32);
-#undef MOE_TOPK_CASE
+  if (S <= 1) launch_topk<1>(nb, hist_smem, s, z, T, E, k, topk_idx, topk_w, block_counts, err);
+  else if (S <= 2) launch_topk<2>(nb, hist_smem, s, z, T, E, k, topk_idx, topk_w, block_counts, err);
+  else if (S <= 4) launch_topk<4>(nb, hist_smem, s, z, T, E, k, topk_idx, topk_w, block_counts, err);
+  else if (S <= 8) launch_topk<8>(nb, hist_smem, s, z, T, E, k, topk_idx, topk_w, block_counts, err);
+  else if (S <= 16) launch_topk<16>(nb, hist_smem, s, z, T, E, k, topk_idx, topk_w, block_counts, err);
+  else launch_topk<32>(nb, hist_smem, s, z, T, E, k, topk_idx, topk_w, block_counts, err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   route_scan_kernel<<<1, 1024, 0, s>>>(block_counts, nb, E, G, block_base, counts, offsets,
