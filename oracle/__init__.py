@@ -75,6 +75,8 @@ def _declare(L):
     L.orc_wgrad_columns.argtypes = [_p, _p, _p, _i64, _p, _p, _p, _i32, _i32, _p, _i32,
                                     _p, _p, _p]
     L.orc_num_threads.restype = _i32
+    L.orc_aux_loss.argtypes = [_p, _p, _i64, _i32, _i32, ctypes.c_double, _p, _p, _p]
+    L.orc_aux_loss_bwd.argtypes = [_p, _p, _i64, _i32, _i32, ctypes.c_double, ctypes.c_double, _p]
 
 
 def _c(a: np.ndarray, dtype) -> np.ndarray:
@@ -224,6 +226,28 @@ def router_bwd(x, Wr, dz, dX, dWr=None, db=None):
     return dX, dWr, db
 
 
+# ------------------------------------------- auxiliary load-balancing loss
+
+def aux_loss(z, counts, k: int, alpha: float):
+    """Switch-style balance loss and routing metrics (orc_aux_loss).
+    Returns dict(importance [E], loss, entropy)."""
+    z = _c(z, np.float64); counts = _c(counts, np.int32)
+    T, E = z.shape
+    imp = np.zeros(E)
+    loss = np.zeros(1); ent = np.zeros(1)
+    lib().orc_aux_loss(_ptr(z), _ptr(counts), T, E, k, float(alpha), _ptr(imp), _ptr(loss), _ptr(ent))
+    return dict(importance=imp, loss=float(loss[0]), entropy=float(ent[0]))
+
+
+def aux_loss_bwd(z, counts, k: int, alpha: float, dL: float = 1.0) -> np.ndarray:
+    """Gradient of the balance loss in the logits, counts held fixed (orc_aux_loss_bwd)."""
+    z = _c(z, np.float64); counts = _c(counts, np.int32)
+    T, E = z.shape
+    dz = np.zeros((T, E))
+    lib().orc_aux_loss_bwd(_ptr(z), _ptr(counts), T, E, k, float(alpha), float(dL), _ptr(dz))
+    return dz
+
+
 # ------------------------------------------------- per-token brute force
 
 def tokens_fwd(xs, idx, w, Wg, Wu, Wd):
@@ -287,12 +311,17 @@ def layer_forward(x, Wr, b, Wg, Wu, Wd, k: int, G: int = 1, logits: str = "f32")
     return dict(z=z, idx=idx, w=w, flags=flags, xp=xp, h1=h1, h2=h2, a=a, yp=yp, Y=Y, **lay)
 
 
-def layer_backward(fw, x, dY, Wr, Wg, Wu, Wd, k: int, acc: Optional[dict] = None):
-    """Whole backward given the forward record `fw` and dY; dW terms add to `acc`."""
+def layer_backward(fw, x, dY, Wr, Wg, Wu, Wd, k: int, acc: Optional[dict] = None,
+                   aux: Optional[tuple] = None):
+    """Whole backward given the forward record `fw` and dY; dW terms add to `acc`.
+    aux = (alpha, dL) adds the balance loss's gradient (dL times dL_aux/dz) to
+    the router's."""
     T = x.shape[0]
     E = Wr.shape[0]
     dyp, dg = combine_bwd(dY, fw["yp"], fw["w"], fw["row_of_pair"])
     dz = route_bwd(dg, fw["w"], fw["idx"], E)
+    if aux is not None:
+        dz = dz + aux_loss_bwd(fw["z"], fw["counts"], k, aux[0], aux[1])
     acc = acc or {}
     dxp, dWg, dWu, dWd = expert_ffn_bwd(fw["xp"], Wg, Wu, Wd, fw["h1"], fw["h2"], fw["a"], dyp,
                                         fw["offsets"], acc.get("dWg"), acc.get("dWu"), acc.get("dWd"))

@@ -378,6 +378,74 @@ void orc_router_bwd(const double* x, const double* Wr, const double* dz,
   }
 }
 
+/* ----------------------------------------- auxiliary load-balancing loss */
+
+/* Auxiliary load-balancing loss and routing metrics. The pages name MoE
+ * losses and metrics without a formula (leap-finetune PR #26 "Add MoE expert
+ * parallel training runtime", its MoE-loss tests); the plainest reading is the
+ * Switch-Transformer balance loss:
+ *   p[t,e] = softmax over all E experts of z[t,:]
+ *   f_e    = counts[e] / (T k)          (fraction of routed pairs to e)
+ *   P_e    = (1/T) sum_t p[t,e]         (importance)
+ *   L      = alpha * E * sum_e f_e P_e
+ *   H      = (1/T) sum_t (- sum_e p[t,e] ln p[t,e]),  0 ln 0 = 0
+ *                                        (mean routing entropy)
+ * f is a count, constant in z. Sums are sequential in t and e. */
+static void orc_softmax_row(const double* z, int E, double* p) {
+  double m = z[0];
+  for (int e = 1; e < E; ++e)
+    if (z[e] > m) m = z[e];
+  double s = 0.0;
+  for (int e = 0; e < E; ++e) {
+    p[e] = exp(z[e] - m);
+    s += p[e];
+  }
+  for (int e = 0; e < E; ++e) p[e] /= s;
+}
+
+void orc_aux_loss(const double* z, const int32_t* counts, int64_t T, int E, int k, double alpha,
+                  double* importance, double* loss, double* entropy) {
+  double* p = (double*)malloc(sizeof(double) * (size_t)E);
+  double h = 0.0;
+  for (int e = 0; e < E; ++e) importance[e] = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    orc_softmax_row(z + t * E, E, p);
+    for (int e = 0; e < E; ++e) {
+      importance[e] += p[e];
+      if (p[e] > 0.0) h -= p[e] * log(p[e]);
+    }
+  }
+  double l = 0.0;
+  for (int e = 0; e < E; ++e) {
+    importance[e] = T > 0 ? importance[e] / (double)T : 0.0;
+    const double fe = T > 0 ? (double)counts[e] / ((double)T * k) : 0.0;
+    l += fe * importance[e];
+  }
+  *loss = alpha * E * l;
+  *entropy = T > 0 ? h / (double)T : 0.0;
+  free(p);
+}
+
+/* Gradient of the loss in z, f held constant (softmax Jacobian):
+ *   dz[t,j] = dL * alpha * E / T * p[t,j] * (f_j - sum_e f_e p[t,e]). */
+void orc_aux_loss_bwd(const double* z, const int32_t* counts, int64_t T, int E, int k,
+                      double alpha, double dL, double* dz) {
+#pragma omp parallel
+  {
+    double* p = (double*)malloc(sizeof(double) * (size_t)E);
+#pragma omp for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+      orc_softmax_row(z + t * E, E, p);
+      double s = 0.0;
+      for (int e = 0; e < E; ++e) s += ((double)counts[e] / ((double)T * k)) * p[e];
+      const double c = dL * alpha * E / (double)T;
+      for (int j = 0; j < E; ++j)
+        dz[t * E + j] = c * p[j] * ((double)counts[j] / ((double)T * k) - s);
+    }
+    free(p);
+  }
+}
+
 /* ------------------------------------------- per-token brute force path */
 
 /* The layer for a list of tokens, evaluated token by token with no

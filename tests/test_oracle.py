@@ -382,3 +382,101 @@ def test_planted_mistakes_are_caught(rng):
     # a permutation off by one row
     bad_rop = np.roll(fw["row_of_pair"], 1)
     assert not np.allclose(oracle.combine(fw["yp"], fw["w"], bad_rop), Y)
+
+
+# ------------------------------------------- auxiliary load-balancing loss
+
+@pytest.mark.parametrize("E,k", [(4, 2), (8, 1), (64, 8)])
+def test_aux_loss_uniform_routing_closed_form(E, k):
+    """Equal logits and equal counts: importance 1/E, loss alpha, entropy ln E."""
+    T = 6 * E
+    z = np.zeros((T, E))
+    counts = np.full(E, T * k // E, np.int32)
+    out = oracle.aux_loss(z, counts, k, 0.02)
+    assert np.allclose(out["importance"], 1.0 / E, rtol=0, atol=1e-15)
+    assert abs(out["loss"] - 0.02) < 1e-15
+    assert abs(out["entropy"] - math.log(E)) < 1e-12
+
+
+def test_aux_loss_collapsed_routing_closed_form():
+    """Every token sends its only pair to expert 0 and its softmax is (almost)
+    one-hot there: the loss reaches its maximum alpha * E and the entropy 0."""
+    T, E = 9, 5
+    z = np.zeros((T, E))
+    z[:, 0] = 60.0
+    counts = np.array([T, 0, 0, 0, 0], np.int32)
+    out = oracle.aux_loss(z, counts, 1, 0.5)
+    p0 = 1.0 / (1.0 + (E - 1) * math.exp(-60.0))
+    assert abs(out["loss"] - 0.5 * E * p0) < 1e-14
+    assert out["entropy"] < 1e-20
+
+
+def test_aux_loss_matches_scipy_softmax_and_entropy(rng):
+    from scipy.special import softmax
+    from scipy.stats import entropy
+    T, E, k = 37, 12, 3
+    z = rng.standard_normal((T, E)) * 2.0
+    counts = rng.integers(0, 20, E).astype(np.int32)
+    out = oracle.aux_loss(z, counts, k, 0.01)
+    p = softmax(z, axis=1)
+    P = p.mean(axis=0)
+    f = counts / (T * k)
+    assert np.allclose(out["importance"], P, rtol=1e-13, atol=0)
+    assert abs(out["loss"] - 0.01 * E * float(np.dot(f, P))) < 1e-15
+    assert abs(out["entropy"] - float(np.mean(entropy(p, axis=1)))) < 1e-12
+
+
+def test_aux_loss_gradient_matches_central_finite_differences(rng):
+    T, E, k, alpha, dL = 5, 6, 2, 0.3, 1.7
+    z = rng.standard_normal((T, E))
+    counts = rng.integers(1, 9, E).astype(np.int32)
+    dz = oracle.aux_loss_bwd(z, counts, k, alpha, dL)
+    h = 1e-6
+    num = np.zeros_like(z)
+    for t in range(T):
+        for e in range(E):
+            zp = z.copy(); zp[t, e] += h
+            zm = z.copy(); zm[t, e] -= h
+            num[t, e] = dL * (oracle.aux_loss(zp, counts, k, alpha)["loss"] -
+                              oracle.aux_loss(zm, counts, k, alpha)["loss"]) / (2 * h)
+    assert np.abs(dz - num).max() <= 1e-7 * np.abs(num).max()
+    # a softmax gradient: every token's row sums to zero
+    assert np.abs(dz.sum(axis=1)).max() < 1e-15
+
+
+def test_aux_loss_router_gradient_matches_finite_differences(rng):
+    """The balance loss composed with z = x Wr^T + b: its gradient through the
+    dense router backward matches central differences in x, Wr and b."""
+    T, d, E, k, alpha = 4, 5, 6, 2, 0.7
+    x = rng.standard_normal((T, d))
+    Wr = rng.standard_normal((E, d)) * 0.5
+    b = rng.standard_normal(E) * 0.3
+    counts = rng.integers(1, 5, E).astype(np.int32)
+
+    def loss(x_, Wr_, b_):
+        return oracle.aux_loss(oracle.router_logits_f64(x_, Wr_, b_), counts, k, alpha)["loss"]
+
+    dz = oracle.aux_loss_bwd(oracle.router_logits_f64(x, Wr, b), counts, k, alpha)
+    dX, dWr, db = oracle.router_bwd(x, Wr, dz, np.zeros((T, d)))
+    h = 1e-6
+    for arr, grad in ((x, dX), (Wr, dWr), (b, db)):
+        num = np.zeros_like(arr)
+        flat = arr.reshape(-1)
+        for i in range(flat.size):
+            old = flat[i]
+            flat[i] = old + h; lp = loss(x, Wr, b)
+            flat[i] = old - h; lm = loss(x, Wr, b)
+            flat[i] = old
+            num.reshape(-1)[i] = (lp - lm) / (2 * h)
+        assert np.abs(grad - num).max() <= 1e-6 * max(np.abs(num).max(), 1e-12)
+
+
+def test_aux_loss_planted_mistake_is_caught():
+    """Counting the fraction per token instead of per routed pair (dropping k)
+    breaks the uniform closed form."""
+    T, E, k = 24, 4, 2
+    z = np.zeros((T, E))
+    counts = np.full(E, T * k // E, np.int32)
+    good = oracle.aux_loss(z, counts, k, 1.0)["loss"]
+    bad = oracle.aux_loss(z, counts, 1, 1.0)["loss"]  # k dropped from f's denominator
+    assert abs(good - 1.0) < 1e-15 and abs(bad - 1.0) > 0.5
