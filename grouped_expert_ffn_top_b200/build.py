@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 
-SOURCES = ["api.cu", "route.cu", "route_noalloc.cu", "dispatch.cu", "grouped_gemm_sm100.cu",
+SOURCES = ["api.cu", "route.cu", "route_noalloc.cu", "aux_loss.cu", "dispatch.cu", "grouped_gemm_sm100.cu",
            "grouped_simt.cu"]
 HEADERS = ["common.cuh", "sm100.cuh", "kernels.h"]
 

@@ -283,6 +283,83 @@ int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_
 
 // ------------------------------------------------------------ grouped FFN
 
+// --------------------------------------------------- auxiliary balance loss
+
+size_t moe_aux_loss_workspace_bytes(int64_t T, int E) {
+  if (T < 0 || E < 1) return 0;
+  return moe::kWsHeader + align256(sizeof(float) * static_cast<size_t>(moe::aux_blocks(T)) * (E + 1));
+}
+
+int moe_aux_loss(const float* logits, const int32_t* expert_counts, int64_t T, int E, int k,
+                 float alpha, float* importance, float* loss, float* entropy, void* ws,
+                 size_t ws_bytes, cudaStream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E)
+    return fail(MOE_ERR_INVALID_ARG, "moe_aux_loss: T=%lld E=%d k=%d", static_cast<long long>(T), E, k);
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_aux_loss: E=%d", E);
+  if (!importance || !loss) return fail(MOE_ERR_INVALID_ARG, "moe_aux_loss: null pointer");
+  if (T == 0) {
+    cudaError_t e = cudaMemsetAsync(importance, 0, sizeof(float) * E, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(loss, 0, sizeof(float), stream);
+    if (e == cudaSuccess && entropy) e = cudaMemsetAsync(entropy, 0, sizeof(float), stream);
+    return cuda_status(e, "moe_aux_loss");
+  }
+  if (!logits || !expert_counts || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_aux_loss: null pointer");
+  if (ws_bytes < moe_aux_loss_workspace_bytes(T, E) || !aligned16(ws))
+    return fail(MOE_ERR_WORKSPACE, "moe_aux_loss: workspace needs %zu bytes (16-byte aligned)",
+                moe_aux_loss_workspace_bytes(T, E));
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + moe::kWsHeader);
+  return launched(cuda_status(moe::launch_aux_loss(logits, expert_counts, T, E, k, alpha,
+                                                   importance, loss, entropy, partial, stream),
+                              "moe_aux_loss"), 2);
+}
+
+int moe_aux_loss_bwd(const float* logits, const int32_t* expert_counts, int64_t T, int E, int k,
+                     float alpha, float dloss, float* dlogits_aux, cudaStream_t stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E)
+    return fail(MOE_ERR_INVALID_ARG, "moe_aux_loss_bwd: T=%lld E=%d k=%d", static_cast<long long>(T), E, k);
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_aux_loss_bwd: E=%d", E);
+  if (T == 0) return MOE_OK;
+  if (!logits || !expert_counts || !dlogits_aux)
+    return fail(MOE_ERR_INVALID_ARG, "moe_aux_loss_bwd: null pointer");
+  return launched(cuda_status(moe::launch_aux_loss_bwd(logits, expert_counts, T, E, k, alpha, dloss,
+                                                       dlogits_aux, stream),
+                              "moe_aux_loss_bwd"), 1);
+}
+
+size_t moe_router_bwd_dense_workspace_bytes(int64_t T, int d, int E) {
+  if (T < 0 || d < 1 || E < 1) return 0;
+  const size_t chunks = static_cast<size_t>(moe::dense_router_chunks(T));
+  return moe::kWsHeader + align256(sizeof(float) * chunks * E * (static_cast<size_t>(d) + 1));
+}
+
+int moe_router_bwd_dense(const void* x, const void* Wr, const float* dz, int dtype, int64_t T,
+                         int d, int E, void* dX, float* dWr, float* db, int accumulate, void* ws,
+                         size_t ws_bytes, cudaStream_t stream) {
+  if (!dtype_ok(dtype)) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd_dense: dtype %d", dtype);
+  if (T < 0 || d < 1 || E < 1)
+    return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd_dense: T=%lld d=%d E=%d",
+                static_cast<long long>(T), d, E);
+  if (d % 4 != 0) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd_dense: d=%d (multiple of 4)", d);
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd_dense: E=%d", E);
+  if (accumulate != 0 && accumulate != 1)
+    return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd_dense: accumulate=%d (0 or 1)", accumulate);
+  if (!dWr) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd_dense: null pointer");
+  if (T == 0) {
+    if (accumulate) return MOE_OK;
+    return cuda_status(zero_grads(stream, sizeof(float) * static_cast<size_t>(E) * d, dWr,
+                                  sizeof(float) * E, db),
+                       "moe_router_bwd_dense");
+  }
+  if (!x || !Wr || !dz || !ws) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd_dense: null pointer");
+  if (ws_bytes < moe_router_bwd_dense_workspace_bytes(T, d, E) || !aligned16(ws))
+    return fail(MOE_ERR_WORKSPACE, "moe_router_bwd_dense: workspace needs %zu bytes (16-byte aligned)",
+                moe_router_bwd_dense_workspace_bytes(T, d, E));
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + moe::kWsHeader);
+  return launched(cuda_status(moe::launch_router_bwd_dense(x, Wr, dz, dtype, T, d, E, dX, dWr, db,
+                                                           accumulate, partial, stream),
+                              "moe_router_bwd_dense"), dX ? 3 : 2);
+}
+
 size_t moe_grouped_ffn_fwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype) {
   (void)rows; (void)E; (void)d; (void)f; (void)dtype;
   return moe::kWsHeader;

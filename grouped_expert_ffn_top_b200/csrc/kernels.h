@@ -65,6 +65,18 @@ struct FfnBwdArgs {
 };
 
 cudaError_t launch_selftest_wait_timeout(unsigned* err, long long limit, cudaStream_t s);
+
+// Auxiliary load-balancing loss (aux_loss.cu).
+int aux_blocks(int64_t T);                 // per-block partials of the forward
+int dense_router_chunks(int64_t T);        // token chunks of the dense router backward
+cudaError_t launch_aux_loss(const float* z, const int32_t* counts, int64_t T, int E, int k,
+                            float alpha, float* importance, float* loss, float* entropy,
+                            float* partial, cudaStream_t s);  // 2 launches
+cudaError_t launch_aux_loss_bwd(const float* z, const int32_t* counts, int64_t T, int E, int k,
+                                float alpha, float dloss, float* dz, cudaStream_t s);  // 1 launch
+cudaError_t launch_router_bwd_dense(const void* x, const void* Wr, const float* dz, int dtype,
+                                    int64_t T, int d, int E, void* dX, float* dWr, float* db,
+                                    int accumulate, float* partial, cudaStream_t s);  // 2 or 3
 cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 2 launches
 cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 1 launch

@@ -5,6 +5,9 @@ Forward:  moe_router_logits -> moe_route -> moe_permute -> moe_grouped_ffn_fwd
 Backward: moe_unpermute_combine_bwd -> moe_route_bwd -> moe_grouped_ffn_dgrad
           -> moe_grouped_ffn_wgrad -> moe_permute_bwd (with the router's input
           gradient) -> moe_router_bwd
+With a balance-loss coefficient (aux_coef > 0) the forward also calls
+moe_aux_loss after routing, and the backward ends with moe_aux_loss_bwd ->
+moe_router_bwd_dense (the loss's dense logit gradient into dX, dWr, db).
 
 The object owns device buffers sized for `max_tokens`, so a step allocates
 nothing; microbatches of any size up to that (0 included) reuse them. Weight
@@ -29,13 +32,13 @@ def _no_mark(name: str) -> None:
 LAUNCHES_PER_CALL = {
     "router_logits": 1, "route": 3, "permute": 1, "grouped_ffn_fwd": 2, "unpermute_combine": 1,
     "unpermute_combine_bwd": 1, "route_bwd": 1, "grouped_ffn_dgrad": 2, "grouped_ffn_wgrad": 1,
-    "permute_bwd": 1, "router_bwd": 2,
+    "permute_bwd": 1, "router_bwd": 2, "aux_loss": 2, "aux_loss_bwd": 1, "router_bwd_dense": 3,
 }
 
 
 class MoELayer:
     def __init__(self, params: Dict[str, torch.Tensor], k: int, ep_groups: int = 1,
-                 max_tokens: int = 0):
+                 max_tokens: int = 0, aux_coef: float = 0.0):
         self.Wr, self.b = params["Wr"], params["b"]
         self.Wg, self.Wu, self.Wd = params["Wg"], params["Wu"], params["Wd"]
         self.E, self.f, self.d = self.Wg.shape
@@ -51,6 +54,14 @@ class MoELayer:
             "dWg": torch.zeros((self.E, self.f, self.d), dtype=f32, device=dev),
             "dWu": torch.zeros((self.E, self.f, self.d), dtype=f32, device=dev),
             "dWd": torch.zeros((self.E, self.d, self.f), dtype=f32, device=dev),
+        }
+        # Switch-style balance loss coefficient (0: no auxiliary loss); after a
+        # forward, self.aux holds its loss [1], importance [E], entropy [1]
+        self.aux_coef = float(aux_coef)
+        self.aux = {
+            "loss": torch.zeros(1, dtype=f32, device=dev),
+            "importance": torch.zeros(self.E, dtype=f32, device=dev),
+            "entropy": torch.zeros(1, dtype=f32, device=dev),
         }
         self.max_tokens = 0
         self.T = 0
@@ -86,6 +97,10 @@ class MoELayer:
             "ffn_bwd": N._ws(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt), dev),
             "router_bwd": N._ws(N.moe_router_bwd_workspace_bytes(P, d, E), dev),
         }
+        if self.aux_coef:
+            self.buf["dz_aux"] = torch.empty((T, E), dtype=f32, device=dev)
+            self.ws["aux"] = N._ws(N.moe_aux_loss_workspace_bytes(T, E), dev)
+            self.ws["dense"] = N._ws(N.moe_router_bwd_dense_workspace_bytes(T, d, E), dev)
         self.max_tokens = T
 
     def zero_grad(self) -> None:
@@ -96,7 +111,7 @@ class MoELayer:
         P = T * self.k
         b = self.buf
         r = self.route
-        v = {n: b[n][:T] for n in ("logits", "Y", "dg", "dlogits", "dX")}
+        v = {n: b[n][:T] for n in ("logits", "Y", "dg", "dlogits", "dX", "dz_aux") if n in b}
         v.update({n: b[n][:P] for n in ("xp", "h1", "h2", "a", "yp", "dyp", "dxp", "dh1", "dh2")})
         ro = dict(r)
         for n in ("topk_idx", "topk_w"):
@@ -120,6 +135,10 @@ class MoELayer:
         mark("router_logits")
         N.moe_route(v["logits"], self.k, self.G, r, self.ws["route"], stream)
         mark("route")
+        if self.aux_coef:
+            N.moe_aux_loss(v["logits"], r["counts"], self.k, self.aux_coef, self.aux, self.ws["aux"],
+                           stream)
+            mark("aux_loss")
         N.moe_permute(x, r["row_of_pair"], self.k, v["xp"], stream)
         mark("permute")
         N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"],
@@ -131,10 +150,11 @@ class MoELayer:
         return Y
 
     def backward(self, dY: torch.Tensor, stream=None, mark=None, out=None,
-                 accumulate: bool = True) -> torch.Tensor:
+                 accumulate: bool = True, aux_dloss: float = 1.0) -> torch.Tensor:
         """dX for upstream gradient dY of the last forward (written to `out`
         if given); dW += the batch's gradient (fp32), or dW = it if not
-        `accumulate`."""
+        `accumulate`. With a balance loss, its gradient (scaled by
+        `aux_dloss`) is included."""
         mark = mark or _no_mark
         T = self.T
         v, r = self.v, self.r
@@ -156,6 +176,13 @@ class MoELayer:
         N.moe_router_bwd(v["xp"], v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"], g["db"],
                          self.ws["router_bwd"], stream, accumulate=accumulate)
         mark("router_bwd")
+        if self.aux_coef:
+            N.moe_aux_loss_bwd(v["logits"], r["counts"], self.k, self.aux_coef, aux_dloss, v["dz_aux"],
+                               stream)
+            mark("aux_loss_bwd")
+            N.moe_router_bwd_dense(self.x, self.Wr, v["dz_aux"], dX, g["dWr"], g["db"], accumulate=True,
+                                   ws=self.ws["dense"], stream=stream)
+            mark("router_bwd_dense")
         return dX
 
     def device_errors(self) -> int:

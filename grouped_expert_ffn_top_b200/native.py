@@ -42,6 +42,7 @@ _p = ctypes.c_void_p
 _i = ctypes.c_int
 _i64 = ctypes.c_int64
 _sz = ctypes.c_size_t
+_f = ctypes.c_float
 
 _SIGNATURES = {
     "moe_last_error": ([], ctypes.c_char_p),
@@ -66,6 +67,11 @@ _SIGNATURES = {
     "moe_permute_bwd": ([_p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p], _i),
     "moe_router_bwd_workspace_bytes": ([_i64, _i, _i], _sz),
     "moe_router_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p, _i, _p, _sz, _p], _i),
+    "moe_aux_loss_workspace_bytes": ([_i64, _i], _sz),
+    "moe_aux_loss": ([_p, _p, _i64, _i, _i, _f, _p, _p, _p, _p, _sz, _p], _i),
+    "moe_aux_loss_bwd": ([_p, _p, _i64, _i, _i, _f, _f, _p, _p], _i),
+    "moe_router_bwd_dense_workspace_bytes": ([_i64, _i, _i], _sz),
+    "moe_router_bwd_dense": ([_p, _p, _p, _i, _i64, _i, _i, _p, _p, _p, _i, _p, _sz, _p], _i),
 }
 
 
@@ -242,6 +248,54 @@ def moe_route_bwd(dg, topk_w, topk_idx, E: int, dlogits=None, stream=None):
     _check(lib().moe_route_bwd(_ptr(dg), _ptr(topk_w), _ptr(topk_idx), T, E, k, _ptr(dlogits),
                                _stream(stream)), "moe_route_bwd")
     return dlogits
+
+
+def moe_aux_loss_workspace_bytes(T, E) -> int:
+    return lib().moe_aux_loss_workspace_bytes(T, E)
+
+
+def moe_aux_loss(logits, expert_counts, k: int, alpha: float, out=None, ws=None, stream=None):
+    """Balance loss and routing metrics; returns dict(importance [E], loss [1], entropy [1])."""
+    _contig(logits, expert_counts)
+    T, E = logits.shape
+    dev = logits.device
+    o = out if out is not None else {
+        "importance": torch.empty(E, dtype=torch.float32, device=dev),
+        "loss": torch.empty(1, dtype=torch.float32, device=dev),
+        "entropy": torch.empty(1, dtype=torch.float32, device=dev)}
+    if ws is None:
+        ws = _ws(moe_aux_loss_workspace_bytes(T, E), dev)
+    _check(lib().moe_aux_loss(_ptr(logits), _ptr(expert_counts), T, E, k, float(alpha),
+                              _ptr(o["importance"]), _ptr(o["loss"]), _ptr(o["entropy"]), _ptr(ws),
+                              ws.numel(), _stream(stream)), "moe_aux_loss")
+    return o
+
+
+def moe_aux_loss_bwd(logits, expert_counts, k: int, alpha: float, dloss: float = 1.0,
+                     dlogits_aux=None, stream=None):
+    _contig(logits, expert_counts)
+    T, E = logits.shape
+    if dlogits_aux is None:
+        dlogits_aux = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    _check(lib().moe_aux_loss_bwd(_ptr(logits), _ptr(expert_counts), T, E, k, float(alpha), float(dloss),
+                                  _ptr(dlogits_aux), _stream(stream)), "moe_aux_loss_bwd")
+    return dlogits_aux
+
+
+def moe_router_bwd_dense_workspace_bytes(T, d, E) -> int:
+    return lib().moe_router_bwd_dense_workspace_bytes(T, d, E)
+
+
+def moe_router_bwd_dense(x, Wr, dz, dX, dWr, db, accumulate: bool = True, ws=None, stream=None):
+    """dX += dz Wr (dX may be None); dWr (+)= dz^T x; db (+)= column sums of dz."""
+    _contig(x, Wr, dz, dX, dWr, db)
+    T, d = x.shape
+    E = Wr.shape[0]
+    if ws is None:
+        ws = _ws(moe_router_bwd_dense_workspace_bytes(T, d, E), x.device)
+    _check(lib().moe_router_bwd_dense(_ptr(x), _ptr(Wr), _ptr(dz), _dt(x), T, d, E, _ptr(dX), _ptr(dWr),
+                                      _ptr(db), int(accumulate), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_router_bwd_dense")
 
 
 def moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype) -> int:

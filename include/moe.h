@@ -322,6 +322,54 @@ MOE_API int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* 
                            int k, float* dWr, float* db, int accumulate, void* ws,
                            size_t ws_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------
+ * Auxiliary load-balancing loss of the router and routing metrics.
+ * The pages name MoE losses and metrics without a formula (leap-finetune
+ * PR #26 "Add MoE expert parallel training runtime", its MoE-loss tests);
+ * the reading taken is the Switch-style balance loss:
+ *   p[t,e] = softmax over all E experts of logits[t,:]
+ *   f_e    = expert_counts[e] / (T k)      (fraction of routed pairs)
+ *   P_e    = (1/T) sum_t p[t,e]            (importance)
+ *   loss   = alpha * E * sum_e f_e P_e
+ *   entropy = (1/T) sum_t -sum_e p[t,e] ln p[t,e]   (mean routing entropy)
+ * f counts routed pairs and is constant in the logits. Sums run in a fixed
+ * order (deterministic). */
+
+/* Workspace of moe_aux_loss, in bytes: per-block partial sums. */
+MOE_API size_t moe_aux_loss_workspace_bytes(int64_t T, int E);
+
+/* logits [T, E] fp32, expert_counts [E] int32 (moe_route's outputs);
+ * importance [E] fp32, loss [1] fp32, entropy [1] fp32 (may be NULL):
+ * device outputs. T = 0 writes zeros. Errors: MOE_ERR_INVALID_ARG (null
+ * pointers, k < 1, k > E), MOE_ERR_UNSUPPORTED (E > MOE_MAX_EXPERTS). */
+MOE_API int moe_aux_loss(const float* logits, const int32_t* expert_counts, int64_t T, int E,
+                         int k, float alpha, float* importance, float* loss, float* entropy,
+                         void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Gradient of dloss * loss in the logits, the counts held fixed:
+ *   dlogits_aux[t,j] = dloss * alpha * E / T * p[t,j] * (f_j - sum_e f_e p[t,e])
+ * written (not added) to dlogits_aux [T, E] fp32. It is dense: carry it to
+ * x, Wr and b with moe_router_bwd_dense. */
+MOE_API int moe_aux_loss_bwd(const float* logits, const int32_t* expert_counts, int64_t T, int E,
+                             int k, float alpha, float dloss, float* dlogits_aux,
+                             cudaStream_t stream);
+
+/* Workspace of moe_router_bwd_dense, in bytes (per-chunk partial sums of
+ * dWr and db: 4 (E d + E) bytes per 256 tokens). */
+MOE_API size_t moe_router_bwd_dense_workspace_bytes(int64_t T, int d, int E);
+
+/* Router backward for a dense logit gradient dz (for example the balance
+ * loss's; moe_permute_bwd and moe_router_bwd use only the selected columns):
+ *   dX[t,:] += sum_e dz[t,e] Wr[e,:]      (dX in the activation dtype, one
+ *                                          rounding of the fp32 sum; may be NULL)
+ *   dWr[e,:] (+)= sum_t dz[t,e] x[t,:];   db[e] (+)= sum_t dz[t,e]
+ * added (accumulate = 1) or written (accumulate = 0); db may be NULL.
+ *   x [T, d] dtype, Wr [E, d] dtype, dz [T, E] fp32. fp32 sums in a fixed
+ * order. d must be a multiple of 4. */
+MOE_API int moe_router_bwd_dense(const void* x, const void* Wr, const float* dz, int dtype,
+                                 int64_t T, int d, int E, void* dX, float* dWr, float* db,
+                                 int accumulate, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

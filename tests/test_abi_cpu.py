@@ -119,3 +119,21 @@ def test_wgrad_accumulate_flag_errors(L):
     bargs = [null] * 8 + [N.MOE_BF16, null, 0, 4, 128, 128, null, null, null, null]
     assert L.moe_grouped_ffn_bwd(*bargs, 1, null, 0, null) == N.MOE_OK
     assert L.moe_grouped_ffn_bwd(*bargs, 0, null, 0, null) == N.MOE_ERR_INVALID_ARG
+
+
+def test_balance_loss_argument_errors(L):
+    f = ctypes.c_float
+    assert L.moe_aux_loss(null, null, 4, 8, 9, f(0.01), null, null, null, null, 0, null) == \
+        N.MOE_ERR_INVALID_ARG  # k > E
+    assert L.moe_aux_loss(null, null, 4, 2048, 2, f(0.01), null, null, null, null, 0, null) == \
+        N.MOE_ERR_UNSUPPORTED  # E > MOE_MAX_EXPERTS
+    assert L.moe_aux_loss(null, null, 4, 8, 2, f(0.01), null, null, null, null, 0, null) == \
+        N.MOE_ERR_INVALID_ARG  # null outputs
+    assert L.moe_aux_loss_bwd(null, null, 0, 8, 2, f(0.01), f(1.0), null, null) == N.MOE_OK
+    assert L.moe_aux_loss_workspace_bytes(1000, 64) >= 256 + 4 * 4 * 65
+    args = [null, null, null, N.MOE_BF16, 10, 130, 8, null, null, null]
+    assert L.moe_router_bwd_dense(*args, 1, null, 0, null) == N.MOE_ERR_UNSUPPORTED  # d % 4
+    args = [null, null, null, N.MOE_BF16, 0, 128, 8, null, null, null]
+    assert L.moe_router_bwd_dense(*args, 2, null, 0, null) == N.MOE_ERR_INVALID_ARG  # accumulate
+    assert L.moe_router_bwd_dense(*args, 1, null, 0, null) == N.MOE_ERR_INVALID_ARG  # null dWr
+    assert L.moe_router_bwd_dense_workspace_bytes(512, 128, 8) >= 256 + 4 * 2 * 8 * 129
