@@ -364,7 +364,7 @@ def run_native(args, w):
     T = w.T[0]
     params = workloads.make_params(w, device=dev, seed=0)
     batch = workloads.make_batch(w, device=dev, seed=R.batch_seed)
-    layer = MoELayer(params, w.k, w.ep_groups, max_tokens=T)
+    layer = MoELayer(params, w.k, w.ep_groups, max_tokens=T, checkpoint=args.checkpoint)
     stream = torch.cuda.current_stream(dev)
     barrier = R.barrier
     max_over_ranks = R.max_over_ranks
@@ -467,7 +467,8 @@ def run_native(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian activations and weights, Zipf-skewed router bias)",
         "impl": "native",
-        "config": dict(workload_config(w), parallelism=f"dp{world}"),
+        "config": dict(workload_config(w), parallelism=f"dp{world}",
+                       **({"checkpoint": "h1, h2 rebuilt in the backward"} if args.checkpoint else {})),
         "grouped_gemm": {"tflops": round(gemm_tf, 1), "frac_bf16_sustained": round(gemm_tf / bf16_sust, 3),
                          "frac_bf16_burst": round(gemm_tf / bf16_burst, 3)},
         "permute_combine": {"gbs": round(mem_gbs, 1), "frac_hbm": round(mem_gbs / hbm, 3),
@@ -503,6 +504,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="fine_fwdbwd_32k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--checkpoint", action="store_true",
+                    help="activation checkpointing: h1, h2 rebuilt in the backward")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -372,11 +372,11 @@ int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const vo
   int rc = check_ffn("moe_grouped_ffn_fwd", dtype, rows, E, d, f);
   if (rc != MOE_OK) return rc;
   if (rows == 0) return MOE_OK;
-  if (!xp || !Wg || !Wu || !Wd || !expert_offsets || !h1 || !h2 || !a || !yp || !ws)
+  if (!xp || !Wg || !Wu || !Wd || !expert_offsets || !a || !yp || !ws || (!h1) != (!h2))
     return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd: null pointer");
   const void* ptrs[] = {xp, Wg, Wu, Wd, h1, h2, a, yp, ws};
   for (const void* q : ptrs)
-    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd: 16-byte alignment");
+    if (q && !aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd: 16-byte alignment");
   if (ws_bytes < moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dtype))
     return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_fwd: workspace too small");
   moe::FfnFwdArgs args{xp, Wg, Wu, Wd, expert_offsets, rows, E, d, f, h1, h2, a, yp,
@@ -384,6 +384,26 @@ int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const vo
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_fwd_bf16(args, stream)
                                     : moe::launch_ffn_fwd_f32(args, stream);
   return launched(cuda_status(e, "moe_grouped_ffn_fwd"), 2);
+}
+
+int moe_grouped_ffn_recompute(const void* xp, const void* Wg, const void* Wu, int dtype,
+                              const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
+                              void* h1, void* h2, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_ffn("moe_grouped_ffn_recompute", dtype, rows, E, d, f);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!xp || !Wg || !Wu || !expert_offsets || !h1 || !h2 || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_recompute: null pointer");
+  const void* ptrs[] = {xp, Wg, Wu, h1, h2, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_recompute: 16-byte alignment");
+  if (ws_bytes < moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_recompute: workspace too small");
+  moe::FfnFwdArgs args{xp, Wg, Wu, nullptr, expert_offsets, rows, E, d, f, h1, h2, nullptr, nullptr,
+                       static_cast<unsigned*>(ws)};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_gateup_bf16(args, stream)
+                                    : moe::launch_ffn_gateup_f32(args, stream);
+  return launched(cuda_status(e, "moe_grouped_ffn_recompute"), 1);
 }
 
 size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype) {

@@ -411,6 +411,7 @@ __device__ __forceinline__ void epilogue_tma(const Params& p, const Maps& maps, 
       __syncwarp();
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
+        if (!optr[t]) continue;  // an output this launch does not store
         // row `lane`: four 16-byte chunks, chunk j at (j ^ ((lane >> 1) & 3)),
         // the TMA 64-byte swizzle of a 64-byte row
         uint8_t* rowp = b + t * BOX + lane * 64;
@@ -422,13 +423,15 @@ __device__ __forceinline__ void epilogue_tma(const Params& p, const Maps& maps, 
       __syncwarp();
       if (lane == 0) {
 #pragma unroll
-        for (int t = 0; t < NT; ++t) tma_store_2d(omap[t], b + t * BOX, ti.n0 + c, ti.row0 + rbase);
+        for (int t = 0; t < NT; ++t)
+          if (optr[t]) tma_store_2d(omap[t], b + t * BOX, ti.n0 + c, ti.row0 + rbase);
         bulk_commit_group();
       }
       ebuf ^= 1;
     } else if (lane < valid) {
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
+        if (!optr[t]) continue;
         bf16* dst = optr[t] + row * ncols + ti.n0 + c;
         store16_bf16(dst, o[t]);
         store16_bf16(dst + 16, o[t] + 16);
@@ -954,7 +957,10 @@ static cudaError_t launch(const Maps& m, const Params& p, cudaStream_t s) {
 
 }  // namespace gg
 
-cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
+// [h1 | h2] = xp [Wg_e | Wu_e]^T and a = silu(h1) h2; each of h1, h2, a is
+// stored only if its pointer is set (a checkpointed forward keeps only a; its
+// backward recomputes h1 and h2 alone).
+cudaError_t launch_ffn_gateup_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   using namespace gg;
   const uint64_t rows = static_cast<uint64_t>(a.rows), E = a.E, d = a.d, f = a.f;
   Params p{};
@@ -970,11 +976,24 @@ cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   p.o0 = static_cast<bf16*>(a.h1);
   p.o1 = static_cast<bf16*>(a.h2);
   p.o2 = static_cast<bf16*>(a.a);
-  if (!make_store_map(&m1.o0, a.h1, f, rows) || !make_store_map(&m1.o1, a.h2, f, rows) ||
-      !make_store_map(&m1.o2, a.a, f, rows))
+  if ((a.h1 && !make_store_map(&m1.o0, a.h1, f, rows)) ||
+      (a.h2 && !make_store_map(&m1.o1, a.h2, f, rows)) ||
+      (a.a && !make_store_map(&m1.o2, a.a, f, rows)))
     return cudaErrorInvalidValue;
-  cudaError_t e = launch<kFwdGateUp, 256, true>(m1, p, s);
+  return launch<kFwdGateUp, 256, true>(m1, p, s);
+}
+
+cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
+  using namespace gg;
+  const uint64_t rows = static_cast<uint64_t>(a.rows), E = a.E, d = a.d, f = a.f;
+  cudaError_t e = launch_ffn_gateup_bf16(a, s);
   if (e != cudaSuccess) return e;
+  Params p{};
+  p.offsets = a.offsets;
+  p.E = a.E;
+  p.d = a.d;
+  p.f = a.f;
+  p.err = a.err;
   Maps m2{};
   // pairs: each CTA stages 128 of the tile's 256 Wd rows
   if (!make_map(&m2.a0, a.a, f, rows, f, 64, 128) || !make_map(&m2.b0, a.Wd, f, E * d, f, 64, 128))

@@ -37,9 +37,9 @@ __global__ void simt_gateup_kernel(const float* __restrict__ xp, const float* __
     s1 = __fmaf_rn(x[i], g[i], s1);
     s2 = __fmaf_rn(x[i], u[i], s2);
   }
-  h1[id] = s1;
-  h2[id] = s2;
-  a[id] = silu_f(s1) * s2;
+  if (h1) h1[id] = s1;  // any of the three may be skipped (checkpointing)
+  if (h2) h2[id] = s2;
+  if (a) a[id] = silu_f(s1) * s2;
 }
 
 // yp = a Wd_e^T     (one thread per (r, i))
@@ -134,6 +134,14 @@ __global__ void simt_wgrad_kernel(const float* __restrict__ xp, const float* __r
 }
 
 static unsigned blocks_for(int64_t n) { return static_cast<unsigned>((n + 255) / 256); }
+
+cudaError_t launch_ffn_gateup_f32(const FfnFwdArgs& x, cudaStream_t s) {
+  simt_gateup_kernel<<<blocks_for(x.rows * x.f), 256, 0, s>>>(
+      static_cast<const float*>(x.xp), static_cast<const float*>(x.Wg),
+      static_cast<const float*>(x.Wu), x.offsets, x.rows, x.E, x.d, x.f,
+      static_cast<float*>(x.h1), static_cast<float*>(x.h2), static_cast<float*>(x.a));
+  return cudaGetLastError();
+}
 
 cudaError_t launch_ffn_fwd_f32(const FfnFwdArgs& x, cudaStream_t s) {
   const float* xp = static_cast<const float*>(x.xp);

@@ -78,6 +78,9 @@ cudaError_t launch_router_bwd_dense(const void* x, const void* Wr, const float* 
                                     int64_t T, int d, int E, void* dX, float* dWr, float* db,
                                     int accumulate, float* partial, cudaStream_t s);  // 2 or 3
 cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s);
+// The gate/up GEMM alone, storing whichever of h1, h2, a are set (1 launch).
+cudaError_t launch_ffn_gateup_bf16(const FfnFwdArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_gateup_f32(const FfnFwdArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 2 launches
 cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 1 launch
 cudaError_t launch_ffn_fwd_f32(const FfnFwdArgs& a, cudaStream_t s);

@@ -5,6 +5,10 @@ Forward:  moe_router_logits -> moe_route -> moe_permute -> moe_grouped_ffn_fwd
 Backward: moe_unpermute_combine_bwd -> moe_route_bwd -> moe_grouped_ffn_dgrad
           -> moe_grouped_ffn_wgrad -> moe_permute_bwd (with the router's input
           gradient) -> moe_router_bwd
+With checkpoint=True the forward does not store h1 and h2 and the backward
+first rebuilds them with moe_grouped_ffn_recompute (activation checkpointing:
+2 T k f activation elements less to keep between forward and backward, for
+one more gate/up GEMM).
 With a balance-loss coefficient (aux_coef > 0) the forward also calls
 moe_aux_loss after routing, and the backward ends with moe_aux_loss_bwd ->
 moe_router_bwd_dense (the loss's dense logit gradient into dX, dWr, db).
@@ -33,12 +37,13 @@ LAUNCHES_PER_CALL = {
     "router_logits": 1, "route": 3, "permute": 1, "grouped_ffn_fwd": 2, "unpermute_combine": 1,
     "unpermute_combine_bwd": 1, "route_bwd": 1, "grouped_ffn_dgrad": 2, "grouped_ffn_wgrad": 1,
     "permute_bwd": 1, "router_bwd": 2, "aux_loss": 2, "aux_loss_bwd": 1, "router_bwd_dense": 3,
+    "grouped_ffn_recompute": 1,
 }
 
 
 class MoELayer:
     def __init__(self, params: Dict[str, torch.Tensor], k: int, ep_groups: int = 1,
-                 max_tokens: int = 0, aux_coef: float = 0.0):
+                 max_tokens: int = 0, aux_coef: float = 0.0, checkpoint: bool = False):
         self.Wr, self.b = params["Wr"], params["b"]
         self.Wg, self.Wu, self.Wd = params["Wg"], params["Wu"], params["Wd"]
         self.E, self.f, self.d = self.Wg.shape
@@ -58,6 +63,7 @@ class MoELayer:
         # Switch-style balance loss coefficient (0: no auxiliary loss); after a
         # forward, self.aux holds its loss [1], importance [E], entropy [1]
         self.aux_coef = float(aux_coef)
+        self.checkpoint = bool(checkpoint)
         self.aux = {
             "loss": torch.zeros(1, dtype=f32, device=dev),
             "importance": torch.zeros(self.E, dtype=f32, device=dev),
@@ -141,8 +147,11 @@ class MoELayer:
             mark("aux_loss")
         N.moe_permute(x, r["row_of_pair"], self.k, v["xp"], stream)
         mark("permute")
-        N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"],
-                              {n: v[n] for n in ("h1", "h2", "a", "yp")}, self.ws["ffn_fwd"], stream)
+        saved = {n: v[n] for n in ("h1", "h2", "a", "yp")}
+        if self.checkpoint:
+            saved["h1"] = saved["h2"] = None  # rebuilt in the backward
+        N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"], saved, self.ws["ffn_fwd"],
+                              stream)
         mark("grouped_ffn_fwd")
         Y = v["Y"] if out is None else out
         N.moe_unpermute_combine(v["yp"], r["topk_w"], r["row_of_pair"], Y, stream)
@@ -163,6 +172,10 @@ class MoELayer:
         mark("unpermute_combine_bwd")
         N.moe_route_bwd(v["dg"], r["topk_w"], r["topk_idx"], self.E, v["dlogits"], stream)
         mark("route_bwd")
+        if self.checkpoint:
+            N.moe_grouped_ffn_recompute(v["xp"], self.Wg, self.Wu, r["offsets"], v["h1"], v["h2"],
+                                        self.ws["ffn_bwd"], stream)
+            mark("grouped_ffn_recompute")
         N.moe_grouped_ffn_dgrad(self.Wg, self.Wu, self.Wd, v["h1"], v["h2"], v["dyp"], r["offsets"],
                                 v["dh1"], v["dh2"], v["dxp"], self.ws["ffn_bwd"], stream)
         mark("grouped_ffn_dgrad")

@@ -68,6 +68,7 @@ _SIGNATURES = {
     "moe_router_bwd_workspace_bytes": ([_i64, _i, _i], _sz),
     "moe_router_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p, _i, _p, _sz, _p], _i),
     "moe_aux_loss_workspace_bytes": ([_i64, _i], _sz),
+    "moe_grouped_ffn_recompute": ([_p, _p, _p, _i, _p, _i64, _i, _i, _i, _p, _p, _p, _sz, _p], _i),
     "moe_aux_loss": ([_p, _p, _i64, _i, _i, _f, _p, _p, _p, _p, _sz, _p], _i),
     "moe_aux_loss_bwd": ([_p, _p, _i64, _i, _i, _f, _f, _p, _p], _i),
     "moe_router_bwd_dense_workspace_bytes": ([_i64, _i, _i], _sz),
@@ -213,6 +214,19 @@ def moe_grouped_ffn_fwd(xp, Wg, Wu, Wd, expert_offsets, out=None, ws=None, strea
                                      _ptr(out["yp"]), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_grouped_ffn_fwd")
     return out
+
+
+def moe_grouped_ffn_recompute(xp, Wg, Wu, expert_offsets, h1, h2, ws=None, stream=None):
+    """h1 = xp Wg_e^T, h2 = xp Wu_e^T for a forward that did not store them."""
+    _contig(xp, Wg, Wu, expert_offsets, h1, h2)
+    rows, d = xp.shape
+    E, f, _ = Wg.shape
+    dt = _dt(xp)
+    if ws is None:
+        ws = _ws(moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dt), xp.device)
+    _check(lib().moe_grouped_ffn_recompute(_ptr(xp), _ptr(Wg), _ptr(Wu), dt, _ptr(expert_offsets), rows, E,
+                                           d, f, _ptr(h1), _ptr(h2), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn_recompute")
 
 
 def moe_unpermute_combine(yp, topk_w, row_of_pair, Y=None, stream=None):

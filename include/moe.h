@@ -210,7 +210,10 @@ MOE_API size_t moe_grouped_ffn_fwd_workspace_bytes(int64_t rows, int E, int d, i
  *   xp [rows, d]; Wg, Wu [E, f, d]; Wd [E, d, f]   dtype inputs
  *   expert_offsets [E+1] int64 (from moe_route), expert_offsets[E] == rows
  *   h1, h2, a [rows, f]; yp [rows, d]              dtype outputs
- *     (h1, h2 and a are saved for the backward)
+ *     (h1, h2 and a are saved for the backward; h1 and h2 may both be NULL:
+ *     then they are not stored, 2 rows * f elements less written, and the
+ *     backward rebuilds them with moe_grouped_ffn_recompute; activation
+ *     checkpointing)
  * Errors: INVALID_ARG; UNSUPPORTED (bf16 needs d and f multiples of 64,
  * fp32 needs multiples of 4; E > MOE_MAX_EXPERTS); WORKSPACE. */
 MOE_API int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,
@@ -243,6 +246,16 @@ MOE_API int moe_unpermute_combine_bwd(const void* dY, const void* yp, const floa
  *   dg, topk_w [T, k] fp32; topk_idx [T, k] int32; dlogits [T, E] fp32 output. */
 MOE_API int moe_route_bwd(const float* dg, const float* topk_w, const int32_t* topk_idx,
                   int64_t T, int E, int k, float* dlogits, cudaStream_t stream);
+
+/* Activation checkpointing: recomputes h1 = xp Wg_e^T and h2 = xp Wu_e^T of
+ * a forward that did not store them (the same kernel and order as
+ * moe_grouped_ffn_fwd, so they are bitwise the values it would have stored).
+ * a is not written. Arguments and errors as moe_grouped_ffn_fwd; ws needs
+ * moe_grouped_ffn_fwd_workspace_bytes() bytes. */
+MOE_API int moe_grouped_ffn_recompute(const void* xp, const void* Wg, const void* Wu, int dtype,
+                                      const int64_t* expert_offsets, int64_t rows, int E, int d,
+                                      int f, void* h1, void* h2, void* ws, size_t ws_bytes,
+                                      cudaStream_t stream);
 
 /* Workspace of moe_grouped_ffn_bwd, in bytes (holds dh1 and dh2). */
 MOE_API size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype);

@@ -107,3 +107,34 @@ def test_layer_with_balance_loss_matches_oracle():
     plain.backward(bt["dY"], accumulate=False)
     torch.cuda.synchronize()
     assert not torch.equal(plain.grads["dWr"], layer.grads["dWr"])
+
+
+# ------------------------------------------------ activation checkpointing
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_checkpointed_backward_is_bitwise_the_stored_one(dtype):
+    """checkpoint=True: the forward leaves h1 and h2 unwritten, the backward
+    rebuilds them with the same kernel, and every output and gradient equals
+    the stored-activation path bit for bit."""
+    T, d, E, k, f = (700, 256, 8, 2, 384) if dtype == "bf16" else (200, 64, 4, 2, 128)
+    w = workloads.custom("ckpt", T, d, E, k, f, dtype=dtype, bias=("normal", 0.5), ep_groups=2)
+    p = workloads.make_params(w, device=DEV, seed=6)
+    bt = workloads.make_batch(w, device=DEV, seed=6)
+    ref = MoELayer(p, k, 2, max_tokens=T)
+    ck = MoELayer(p, k, 2, max_tokens=T, checkpoint=True)
+    ck.buf["h1"].fill_(float("nan"))
+    ck.buf["h2"].fill_(float("nan"))
+    Y0 = ref.forward(bt["x"]).clone()
+    Y1 = ck.forward(bt["x"]).clone()
+    torch.cuda.synchronize()
+    assert torch.isnan(ck.buf["h1"]).all() and torch.isnan(ck.buf["h2"]).all()
+    assert torch.equal(Y0, Y1)
+    dX0 = ref.backward(bt["dY"], accumulate=False).clone()
+    dX1 = ck.backward(bt["dY"], accumulate=False).clone()
+    torch.cuda.synchronize()
+    assert ck.device_errors() == 0
+    assert torch.equal(dX0, dX1)
+    for n in ("h1", "h2", "dh1", "dh2"):
+        assert torch.equal(ref.v[n], ck.v[n]), n
+    for n in ref.grads:
+        assert torch.equal(ref.grads[n], ck.grads[n]), n
