@@ -1,0 +1,66 @@
+"""Expert parallelism on one GPU: with one rank the expert-parallel layer's
+exchanges are identities, so through the library's kernels it must give the
+plain layer's results bit for bit, with no process group and through a
+one-rank NCCL group (which runs the real all-to-all calls)."""
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+
+from grouped_expert_ffn_top_b200 import native as N
+from grouped_expert_ffn_top_b200 import workloads
+from grouped_expert_ffn_top_b200.ep import EPMoELayer
+from grouped_expert_ffn_top_b200.layer import MoELayer
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    N.lib()
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _compare(with_group: bool):
+    T, d, E, k, f = 700, 256, 8, 2, 384
+    w = workloads.custom("ep1", T, d, E, k, f, bias=("normal", 0.5))
+    p = workloads.make_params(w, device=DEV, seed=8)
+    p["b"][E - 1] = -1.0e4
+    bt = workloads.make_batch(w, device=DEV, seed=8)
+    ref = MoELayer(p, k, 1, max_tokens=T)
+    Y0 = ref.forward(bt["x"]).clone()
+    dX0 = ref.backward(bt["dY"], accumulate=False).clone()
+    if with_group:
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                                world_size=1)
+    try:
+        ep = EPMoELayer(p, E, k)
+        Y1 = ep.forward(bt["x"])
+        dX1 = ep.backward(bt["dY"], accumulate=False)
+        torch.cuda.synchronize()
+    finally:
+        if with_group:
+            dist.destroy_process_group()
+    assert torch.equal(Y0, Y1)
+    assert torch.equal(dX0, dX1)
+    for n in ref.grads:
+        assert torch.equal(ref.grads[n], ep.grads[n]), n
+
+
+def test_one_rank_expert_parallel_layer_is_the_plain_layer():
+    _compare(with_group=False)
+
+
+def test_one_rank_nccl_expert_parallel_layer_is_the_plain_layer():
+    _compare(with_group=True)
