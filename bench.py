@@ -64,6 +64,9 @@ def algorithmic_work(w, T: int):
         "grouped_ffn_wgrad": 6.0 * d * f * P,
         "router_bwd": 2.0 * T * d * E,
     }
+    # the fused-dispatch forms do the same arithmetic
+    for n in ("grouped_ffn_fwd", "grouped_ffn_wgrad", "router_bwd"):
+        flops[n + "_gather"] = flops[n]
     bytes_ = {
         "permute": (T * d + P * d) * b + 4 * P,
         "unpermute_combine": (P * d + T * d) * b + 8 * P,
@@ -364,7 +367,10 @@ def run_native(args, w):
     T = w.T[0]
     params = workloads.make_params(w, device=dev, seed=0)
     batch = workloads.make_batch(w, device=dev, seed=R.batch_seed)
-    layer = MoELayer(params, w.k, w.ep_groups, max_tokens=T, checkpoint=args.checkpoint)
+    fused = args.dispatch == "fused"
+    sfx = "_gather" if fused else ""
+    layer = MoELayer(params, w.k, w.ep_groups, max_tokens=T, checkpoint=args.checkpoint,
+                     fused_dispatch=fused)
     stream = torch.cuda.current_stream(dev)
     barrier = R.barrier
     max_over_ranks = R.max_over_ranks
@@ -444,17 +450,18 @@ def run_native(args, w):
                         "frac_8tbs": round(gbs / 8000.0, 3)})
         kernels[n] = ent
 
-    wg_ms = call_ms["grouped_ffn_wgrad"]
+    wg_ms = call_ms["grouped_ffn_wgrad" + sfx]
     wg_tf = flops["grouped_ffn_wgrad"] / (wg_ms * 1e-3) / 1e12
-    traffic = ncu_traffic("grouped_ffn_wgrad")
-    roofline = {"kernel": "grouped_ffn_wgrad (tcgen05 grouped GEMM, ragged K)", "bound": "tensor",
+    traffic = ncu_traffic("grouped_ffn_wgrad" + sfx)
+    roofline = {"kernel": f"grouped_ffn_wgrad{sfx} (tcgen05 grouped GEMM, ragged K)", "bound": "tensor",
                 "achieved": round(wg_tf, 1), "peak": bf16_sust, "unit": "TFLOP/s",
                 "frac": round(wg_tf / bf16_sust, 3), "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 sustained (timed inside a long step)",
                 "algorithmic_flops_per_launch": flops["grouped_ffn_wgrad"]}
-    gemm_ms = sum(call_ms[n] for n in ("grouped_ffn_fwd", "grouped_ffn_dgrad", "grouped_ffn_wgrad"))
+    gemm_ms = sum(call_ms[n] for n in ("grouped_ffn_fwd" + sfx, "grouped_ffn_dgrad", "grouped_ffn_wgrad" + sfx))
     gemm_tf = 18.0 * w.d * w.f * T * w.k / (gemm_ms * 1e-3) / 1e12
-    mem_calls = ("permute", "unpermute_combine", "unpermute_combine_bwd", "permute_bwd")
+    mem_calls = tuple(n for n in ("permute", "unpermute_combine", "unpermute_combine_bwd", "permute_bwd")
+                      if n in call_ms)
     mem_ms = sum(call_ms[n] for n in mem_calls)
     mem_gbs = sum(bytes_[n] for n in mem_calls) / (mem_ms * 1e-3) / 1e9
 
@@ -468,7 +475,9 @@ def run_native(args, w):
         "data": "synthetic (seeded Gaussian activations and weights, Zipf-skewed router bias)",
         "impl": "native",
         "config": dict(workload_config(w), parallelism=f"dp{world}",
-                       **({"checkpoint": "h1, h2 rebuilt in the backward"} if args.checkpoint else {})),
+                       **({"checkpoint": "h1, h2 rebuilt in the backward"} if args.checkpoint else {}),
+                       dispatch=("fused: expert rows gathered from x inside the GEMM operand loads, "
+                                 "no permuted copy" if fused else "permute: rows copied to xp first")),
         "grouped_gemm": {"tflops": round(gemm_tf, 1), "frac_bf16_sustained": round(gemm_tf / bf16_sust, 3),
                          "frac_bf16_burst": round(gemm_tf / bf16_burst, 3)},
         "permute_combine": {"gbs": round(mem_gbs, 1), "frac_hbm": round(mem_gbs / hbm, 3),
@@ -506,6 +515,9 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--checkpoint", action="store_true",
                     help="activation checkpointing: h1, h2 rebuilt in the backward")
+    ap.add_argument("--dispatch", choices=["permute", "fused"], default="permute",
+                    help="permute: copy the dispatch rows to xp before the GEMMs; fused: gather them "
+                         "from x inside the GEMMs' operand loads")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

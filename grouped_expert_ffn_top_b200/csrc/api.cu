@@ -251,34 +251,55 @@ size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E) {
   return moe::kWsHeader + align256(sizeof(float) * items * (static_cast<size_t>(d) + 1));
 }
 
-int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_row,
-                   const int64_t* expert_offsets, int dtype, int64_t T, int d, int E, int k,
-                   float* dWr, float* db, int accumulate, void* ws, size_t ws_bytes,
-                   cudaStream_t stream) {
-  int rc = check_rows("moe_router_bwd", dtype, T, d, k);
+}  // extern "C"
+
+// xp, or with `gather` x [T, d] read through pair_of_row
+static int router_bwd_impl(const char* fn, bool gather, const void* xp, const float* dlogits,
+                           const int32_t* pair_of_row, const int64_t* expert_offsets, int dtype,
+                           int64_t T, int d, int E, int k, float* dWr, float* db, int accumulate,
+                           void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_rows(fn, dtype, T, d, k);
   if (rc != MOE_OK) return rc;
-  if (E < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: E=%d k=%d", E, k);
-  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "moe_router_bwd: E=%d", E);
+  if (E < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "%s: E=%d k=%d", fn, E, k);
+  if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "%s: E=%d", fn, E);
   if (accumulate != 0 && accumulate != 1)
-    return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: accumulate=%d (0 or 1)", accumulate);
+    return fail(MOE_ERR_INVALID_ARG, "%s: accumulate=%d (0 or 1)", fn, accumulate);
   if (T == 0) {
     if (accumulate) return MOE_OK;
-    if (!dWr) return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: null pointer");
+    if (!dWr) return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
     return cuda_status(zero_grads(stream, sizeof(float) * static_cast<size_t>(E) * d, dWr,
                                   sizeof(float) * E, db),
-                       "moe_router_bwd");
+                       fn);
   }
   if (!xp || !dlogits || !pair_of_row || !expert_offsets || !dWr || !ws)
-    return fail(MOE_ERR_INVALID_ARG, "moe_router_bwd: null pointer");
+    return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
   const int64_t rows = T * k;
   if (ws_bytes < moe_router_bwd_workspace_bytes(rows, d, E) || !aligned16(ws) || !aligned16(xp))
-    return fail(MOE_ERR_WORKSPACE, "moe_router_bwd: workspace needs %zu bytes (16-byte aligned)",
+    return fail(MOE_ERR_WORKSPACE, "%s: workspace needs %zu bytes (16-byte aligned)", fn,
                 moe_router_bwd_workspace_bytes(rows, d, E));
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + moe::kWsHeader);
   return launched(cuda_status(moe::launch_router_bwd(xp, dlogits, pair_of_row, expert_offsets,
                                                       dtype, rows, d, E, k, dWr, db, accumulate,
-                                                      partial, stream),
-                              "moe_router_bwd"), 2);
+                                                      partial, stream, gather),
+                              fn), 2);
+}
+
+extern "C" {
+
+int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* pair_of_row,
+                   const int64_t* expert_offsets, int dtype, int64_t T, int d, int E, int k,
+                   float* dWr, float* db, int accumulate, void* ws, size_t ws_bytes,
+                   cudaStream_t stream) {
+  return router_bwd_impl("moe_router_bwd", false, xp, dlogits, pair_of_row, expert_offsets, dtype,
+                         T, d, E, k, dWr, db, accumulate, ws, ws_bytes, stream);
+}
+
+int moe_router_bwd_gather(const void* x, const float* dlogits, const int32_t* pair_of_row,
+                          const int64_t* expert_offsets, int dtype, int64_t T, int d, int E, int k,
+                          float* dWr, float* db, int accumulate, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  return router_bwd_impl("moe_router_bwd_gather", true, x, dlogits, pair_of_row, expert_offsets,
+                         dtype, T, d, E, k, dWr, db, accumulate, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------ grouped FFN
@@ -365,45 +386,179 @@ size_t moe_grouped_ffn_fwd_workspace_bytes(int64_t rows, int E, int d, int f, in
   return moe::kWsHeader;
 }
 
+}  // extern "C"
+
+// The expert input of a grouped-FFN call: xp [rows, d], or x [T, d] read
+// through pair_of_row (rows = T k; dispatch row r is x[pair_of_row[r] / k]).
+static int check_gather(const char* fn, const moe::RowGather& g, int dtype, int64_t rows, int d) {
+  if (!g.rows) return MOE_OK;
+  int rc = check_rows(fn, dtype, g.T, d, g.k);
+  if (rc != MOE_OK) return rc;
+  if (g.T * g.k != rows)
+    return fail(MOE_ERR_INVALID_ARG, "%s: rows=%lld != T*k=%lld", fn, static_cast<long long>(rows),
+                static_cast<long long>(g.T * g.k));
+  return MOE_OK;
+}
+
+static int ffn_fwd_impl(const char* fn, const void* xp, const moe::RowGather& g, const void* Wg,
+                        const void* Wu, const void* Wd, int dtype, const int64_t* expert_offsets,
+                        int64_t rows, int E, int d, int f, void* h1, void* h2, void* a, void* yp,
+                        void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_ffn(fn, dtype, rows, E, d, f);
+  if (rc == MOE_OK) rc = check_gather(fn, g, dtype, rows, d);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!xp || !Wg || !Wu || !Wd || !expert_offsets || !a || !yp || !ws || (!h1) != (!h2))
+    return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
+  const void* ptrs[] = {xp, Wg, Wu, Wd, h1, h2, a, yp, ws};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "%s: 16-byte alignment", fn);
+  if (ws_bytes < moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "%s: workspace too small", fn);
+  moe::FfnFwdArgs args{xp, Wg, Wu, Wd, expert_offsets, rows, E, d, f, h1, h2, a, yp,
+                       static_cast<unsigned*>(ws), g};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_fwd_bf16(args, stream)
+                                    : moe::launch_ffn_fwd_f32(args, stream);
+  return launched(cuda_status(e, fn), 2);
+}
+
+static int ffn_recompute_impl(const char* fn, const void* xp, const moe::RowGather& g,
+                              const void* Wg, const void* Wu, int dtype,
+                              const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
+                              void* h1, void* h2, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_ffn(fn, dtype, rows, E, d, f);
+  if (rc == MOE_OK) rc = check_gather(fn, g, dtype, rows, d);
+  if (rc != MOE_OK) return rc;
+  if (rows == 0) return MOE_OK;
+  if (!xp || !Wg || !Wu || !expert_offsets || !h1 || !h2 || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
+  const void* ptrs[] = {xp, Wg, Wu, h1, h2, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "%s: 16-byte alignment", fn);
+  if (ws_bytes < moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "%s: workspace too small", fn);
+  moe::FfnFwdArgs args{xp, Wg, Wu, nullptr, expert_offsets, rows, E, d, f, h1, h2, nullptr, nullptr,
+                       static_cast<unsigned*>(ws), g};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_gateup_bf16(args, stream)
+                                    : moe::launch_ffn_gateup_f32(args, stream);
+  return launched(cuda_status(e, fn), 1);
+}
+
+static int ffn_bwd_impl(const char* fn, const void* xp, const moe::RowGather& g, const void* Wg,
+                        const void* Wu, const void* Wd, const void* h1, const void* h2,
+                        const void* a, const void* dyp, int dtype, const int64_t* expert_offsets,
+                        int64_t rows, int E, int d, int f, void* dxp, float* dWg, float* dWu,
+                        float* dWd, int accumulate, void* ws, size_t ws_bytes,
+                        cudaStream_t stream) {
+  int rc = check_ffn(fn, dtype, rows, E, d, f);
+  if (rc == MOE_OK) rc = check_gather(fn, g, dtype, rows, d);
+  if (rc != MOE_OK) return rc;
+  if (accumulate != 0 && accumulate != 1)
+    return fail(MOE_ERR_INVALID_ARG, "%s: accumulate=%d (0 or 1)", fn, accumulate);
+  if (rows == 0) {
+    if (accumulate) return MOE_OK;
+    if (!dWg || !dWu || !dWd) return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
+    const size_t n = sizeof(float) * static_cast<size_t>(E) * f * d;
+    return cuda_status(zero_grads(stream, n, dWg, n, dWu, n, dWd), fn);
+  }
+  if (!xp || !Wg || !Wu || !Wd || !h1 || !h2 || !a || !dyp || !expert_offsets || !dxp || !dWg ||
+      !dWu || !dWd || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
+  const void* ptrs[] = {xp, Wg, Wu, Wd, h1, h2, a, dyp, dxp, dWg, dWu, dWd, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "%s: 16-byte alignment", fn);
+  if (ws_bytes < moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "%s: workspace needs %zu bytes (got %zu)", fn,
+                moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype), ws_bytes);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t h = align256(static_cast<size_t>(rows) * f * elem_bytes(dtype));
+  moe::FfnBwdArgs args{xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, rows, E, d, f, dxp,
+                       dWg, dWu, dWd, base + moe::kWsHeader, base + moe::kWsHeader + h,
+                       static_cast<unsigned*>(ws), accumulate, g};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
+                                    : moe::launch_ffn_dgrad_f32(args, stream);
+  if (e == cudaSuccess) {
+    counted(2);
+    e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
+                          : moe::launch_ffn_wgrad_f32(args, stream);
+  }
+  return launched(cuda_status(e, fn), 1);
+}
+
+static int ffn_wgrad_impl(const char* fn, const void* xp, const moe::RowGather& g, const void* a,
+                          const void* dyp, const void* dh1, const void* dh2, int dtype,
+                          const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
+                          float* dWg, float* dWu, float* dWd, int accumulate, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+  int rc = check_ffn(fn, dtype, rows, E, d, f);
+  if (rc == MOE_OK) rc = check_gather(fn, g, dtype, rows, d);
+  if (rc != MOE_OK) return rc;
+  if (accumulate != 0 && accumulate != 1)
+    return fail(MOE_ERR_INVALID_ARG, "%s: accumulate=%d (0 or 1)", fn, accumulate);
+  if (rows == 0) {
+    if (accumulate) return MOE_OK;
+    if (!dWg || !dWu || !dWd) return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
+    const size_t n = sizeof(float) * static_cast<size_t>(E) * f * d;
+    return cuda_status(zero_grads(stream, n, dWg, n, dWu, n, dWd), fn);
+  }
+  if (!xp || !a || !dyp || !dh1 || !dh2 || !expert_offsets || !dWg || !dWu || !dWd || !ws)
+    return fail(MOE_ERR_INVALID_ARG, "%s: null pointer", fn);
+  const void* ptrs[] = {xp, a, dyp, dh1, dh2, dWg, dWu, dWd, ws};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "%s: 16-byte alignment", fn);
+  if (ws_bytes < moe::kWsHeader) return fail(MOE_ERR_WORKSPACE, "%s: workspace", fn);
+  moe::FfnBwdArgs args{xp, nullptr, nullptr, nullptr, nullptr, nullptr, a, dyp, expert_offsets,
+                       rows, E, d, f, nullptr, dWg, dWu, dWd, const_cast<void*>(dh1),
+                       const_cast<void*>(dh2), static_cast<unsigned*>(ws), accumulate, g};
+  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
+                                    : moe::launch_ffn_wgrad_f32(args, stream);
+  return launched(cuda_status(e, fn), 1);
+}
+
+static moe::RowGather row_gather(const int32_t* pair_of_row, int64_t T, int k) {
+  moe::RowGather g;
+  g.rows = pair_of_row;
+  g.k = k;
+  g.T = T;
+  return g;
+}
+
+extern "C" {
+
 int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const void* Wd, int dtype,
                         const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
                         void* h1, void* h2, void* a, void* yp, void* ws, size_t ws_bytes,
                         cudaStream_t stream) {
-  int rc = check_ffn("moe_grouped_ffn_fwd", dtype, rows, E, d, f);
-  if (rc != MOE_OK) return rc;
-  if (rows == 0) return MOE_OK;
-  if (!xp || !Wg || !Wu || !Wd || !expert_offsets || !a || !yp || !ws || (!h1) != (!h2))
-    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd: null pointer");
-  const void* ptrs[] = {xp, Wg, Wu, Wd, h1, h2, a, yp, ws};
-  for (const void* q : ptrs)
-    if (q && !aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd: 16-byte alignment");
-  if (ws_bytes < moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dtype))
-    return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_fwd: workspace too small");
-  moe::FfnFwdArgs args{xp, Wg, Wu, Wd, expert_offsets, rows, E, d, f, h1, h2, a, yp,
-                       static_cast<unsigned*>(ws)};
-  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_fwd_bf16(args, stream)
-                                    : moe::launch_ffn_fwd_f32(args, stream);
-  return launched(cuda_status(e, "moe_grouped_ffn_fwd"), 2);
+  return ffn_fwd_impl("moe_grouped_ffn_fwd", xp, moe::RowGather{}, Wg, Wu, Wd, dtype,
+                      expert_offsets, rows, E, d, f, h1, h2, a, yp, ws, ws_bytes, stream);
+}
+
+int moe_grouped_ffn_fwd_gather(const void* x, const int32_t* pair_of_row, int64_t T, int k,
+                               const void* Wg, const void* Wu, const void* Wd, int dtype,
+                               const int64_t* expert_offsets, int E, int d, int f, void* h1,
+                               void* h2, void* a, void* yp, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+  if (!pair_of_row && T > 0) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_fwd_gather: null pointer");
+  return ffn_fwd_impl("moe_grouped_ffn_fwd_gather", x, row_gather(pair_of_row, T, k), Wg, Wu, Wd,
+                      dtype, expert_offsets, T * k, E, d, f, h1, h2, a, yp, ws, ws_bytes, stream);
 }
 
 int moe_grouped_ffn_recompute(const void* xp, const void* Wg, const void* Wu, int dtype,
                               const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
                               void* h1, void* h2, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  int rc = check_ffn("moe_grouped_ffn_recompute", dtype, rows, E, d, f);
-  if (rc != MOE_OK) return rc;
-  if (rows == 0) return MOE_OK;
-  if (!xp || !Wg || !Wu || !expert_offsets || !h1 || !h2 || !ws)
-    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_recompute: null pointer");
-  const void* ptrs[] = {xp, Wg, Wu, h1, h2, ws};
-  for (const void* q : ptrs)
-    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_recompute: 16-byte alignment");
-  if (ws_bytes < moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dtype))
-    return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_recompute: workspace too small");
-  moe::FfnFwdArgs args{xp, Wg, Wu, nullptr, expert_offsets, rows, E, d, f, h1, h2, nullptr, nullptr,
-                       static_cast<unsigned*>(ws)};
-  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_gateup_bf16(args, stream)
-                                    : moe::launch_ffn_gateup_f32(args, stream);
-  return launched(cuda_status(e, "moe_grouped_ffn_recompute"), 1);
+  return ffn_recompute_impl("moe_grouped_ffn_recompute", xp, moe::RowGather{}, Wg, Wu, dtype,
+                            expert_offsets, rows, E, d, f, h1, h2, ws, ws_bytes, stream);
+}
+
+int moe_grouped_ffn_recompute_gather(const void* x, const int32_t* pair_of_row, int64_t T, int k,
+                                     const void* Wg, const void* Wu, int dtype,
+                                     const int64_t* expert_offsets, int E, int d, int f, void* h1,
+                                     void* h2, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!pair_of_row && T > 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_recompute_gather: null pointer");
+  return ffn_recompute_impl("moe_grouped_ffn_recompute_gather", x, row_gather(pair_of_row, T, k),
+                            Wg, Wu, dtype, expert_offsets, T * k, E, d, f, h1, h2, ws, ws_bytes,
+                            stream);
 }
 
 size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype) {
@@ -418,38 +573,21 @@ int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const vo
                         const int64_t* expert_offsets, int64_t rows, int E, int d, int f,
                         void* dxp, float* dWg, float* dWu, float* dWd, int accumulate, void* ws,
                         size_t ws_bytes, cudaStream_t stream) {
-  int rc = check_ffn("moe_grouped_ffn_bwd", dtype, rows, E, d, f);
-  if (rc != MOE_OK) return rc;
-  if (accumulate != 0 && accumulate != 1)
-    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: accumulate=%d (0 or 1)", accumulate);
-  if (rows == 0) {
-    if (accumulate) return MOE_OK;
-    if (!dWg || !dWu || !dWd) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: null pointer");
-    const size_t n = sizeof(float) * static_cast<size_t>(E) * f * d;
-    return cuda_status(zero_grads(stream, n, dWg, n, dWu, n, dWd), "moe_grouped_ffn_bwd");
-  }
-  if (!xp || !Wg || !Wu || !Wd || !h1 || !h2 || !a || !dyp || !expert_offsets || !dxp || !dWg ||
-      !dWu || !dWd || !ws)
-    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: null pointer");
-  const void* ptrs[] = {xp, Wg, Wu, Wd, h1, h2, a, dyp, dxp, dWg, dWu, dWd, ws};
-  for (const void* q : ptrs)
-    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd: 16-byte alignment");
-  if (ws_bytes < moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype))
-    return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_bwd: workspace needs %zu bytes (got %zu)",
-                moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype), ws_bytes);
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  const size_t h = align256(static_cast<size_t>(rows) * f * elem_bytes(dtype));
-  moe::FfnBwdArgs args{xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, rows, E, d, f, dxp,
-                       dWg, dWu, dWd, base + moe::kWsHeader, base + moe::kWsHeader + h,
-                       static_cast<unsigned*>(ws), accumulate};
-  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
-                                    : moe::launch_ffn_dgrad_f32(args, stream);
-  if (e == cudaSuccess) {
-    counted(2);
-    e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
-                          : moe::launch_ffn_wgrad_f32(args, stream);
-  }
-  return launched(cuda_status(e, "moe_grouped_ffn_bwd"), 1);
+  return ffn_bwd_impl("moe_grouped_ffn_bwd", xp, moe::RowGather{}, Wg, Wu, Wd, h1, h2, a, dyp,
+                      dtype, expert_offsets, rows, E, d, f, dxp, dWg, dWu, dWd, accumulate, ws,
+                      ws_bytes, stream);
+}
+
+int moe_grouped_ffn_bwd_gather(const void* x, const int32_t* pair_of_row, int64_t T, int k,
+                               const void* Wg, const void* Wu, const void* Wd, const void* h1,
+                               const void* h2, const void* a, const void* dyp, int dtype,
+                               const int64_t* expert_offsets, int E, int d, int f, void* dxp,
+                               float* dWg, float* dWu, float* dWd, int accumulate, void* ws,
+                               size_t ws_bytes, cudaStream_t stream) {
+  if (!pair_of_row && T > 0) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_bwd_gather: null pointer");
+  return ffn_bwd_impl("moe_grouped_ffn_bwd_gather", x, row_gather(pair_of_row, T, k), Wg, Wu, Wd,
+                      h1, h2, a, dyp, dtype, expert_offsets, T * k, E, d, f, dxp, dWg, dWu, dWd,
+                      accumulate, ws, ws_bytes, stream);
 }
 
 int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const void* h1,
@@ -476,28 +614,21 @@ int moe_grouped_ffn_wgrad(const void* xp, const void* a, const void* dyp, const 
                           const void* dh2, int dtype, const int64_t* expert_offsets, int64_t rows,
                           int E, int d, int f, float* dWg, float* dWu, float* dWd, int accumulate,
                           void* ws, size_t ws_bytes, cudaStream_t stream) {
-  int rc = check_ffn("moe_grouped_ffn_wgrad", dtype, rows, E, d, f);
-  if (rc != MOE_OK) return rc;
-  if (accumulate != 0 && accumulate != 1)
-    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: accumulate=%d (0 or 1)", accumulate);
-  if (rows == 0) {
-    if (accumulate) return MOE_OK;
-    if (!dWg || !dWu || !dWd) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: null pointer");
-    const size_t n = sizeof(float) * static_cast<size_t>(E) * f * d;
-    return cuda_status(zero_grads(stream, n, dWg, n, dWu, n, dWd), "moe_grouped_ffn_wgrad");
-  }
-  if (!xp || !a || !dyp || !dh1 || !dh2 || !expert_offsets || !dWg || !dWu || !dWd || !ws)
-    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: null pointer");
-  const void* ptrs[] = {xp, a, dyp, dh1, dh2, dWg, dWu, dWd, ws};
-  for (const void* q : ptrs)
-    if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad: 16-byte alignment");
-  if (ws_bytes < moe::kWsHeader) return fail(MOE_ERR_WORKSPACE, "moe_grouped_ffn_wgrad: workspace");
-  moe::FfnBwdArgs args{xp, nullptr, nullptr, nullptr, nullptr, nullptr, a, dyp, expert_offsets,
-                       rows, E, d, f, nullptr, dWg, dWu, dWd, const_cast<void*>(dh1),
-                       const_cast<void*>(dh2), static_cast<unsigned*>(ws), accumulate};
-  cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
-                                    : moe::launch_ffn_wgrad_f32(args, stream);
-  return launched(cuda_status(e, "moe_grouped_ffn_wgrad"), 1);
+  return ffn_wgrad_impl("moe_grouped_ffn_wgrad", xp, moe::RowGather{}, a, dyp, dh1, dh2, dtype,
+                        expert_offsets, rows, E, d, f, dWg, dWu, dWd, accumulate, ws, ws_bytes,
+                        stream);
+}
+
+int moe_grouped_ffn_wgrad_gather(const void* x, const int32_t* pair_of_row, int64_t T, int k,
+                                 const void* a, const void* dyp, const void* dh1, const void* dh2,
+                                 int dtype, const int64_t* expert_offsets, int E, int d, int f,
+                                 float* dWg, float* dWu, float* dWd, int accumulate, void* ws,
+                                 size_t ws_bytes, cudaStream_t stream) {
+  if (!pair_of_row && T > 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_grouped_ffn_wgrad_gather: null pointer");
+  return ffn_wgrad_impl("moe_grouped_ffn_wgrad_gather", x, row_gather(pair_of_row, T, k), a, dyp,
+                        dh1, dh2, dtype, expert_offsets, T * k, E, d, f, dWg, dWu, dWd, accumulate,
+                        ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -359,7 +359,9 @@ __device__ __forceinline__ int expert_of_item(const int* s_start, int E, int ite
 // partial[item, cols] = sum over the item's rows r (ascending) of
 // dz[token(r), e] * xp[r, cols]; partial_db[item] = sum of those dz.
 // Each xp row is read once, 16 bytes per thread, coalesced across the block.
-template <typename T>
+// GATHER: `xp` is x [T, d] and row r is read as x[token(r)] (the same values,
+// since xp[r] is a copy of x[token(r)]), so xp need not exist.
+template <typename T, bool GATHER>
 __global__ void __launch_bounds__(kRbThreads) router_wgrad_partial_kernel(
     const T* __restrict__ xp, const float* __restrict__ dz, const int32_t* __restrict__ por,
     const int64_t* __restrict__ off, int E, int d, int k, float* __restrict__ partial,
@@ -367,24 +369,29 @@ __global__ void __launch_bounds__(kRbThreads) router_wgrad_partial_kernel(
   constexpr int VE = Vec16<T>::N;
   __shared__ int s_start[MOE_MAX_EXPERTS + 1];
   __shared__ float s_dz[kRbRows];
+  __shared__ int s_tok[GATHER ? kRbRows : 1];
   router_items_prefix(off, E, s_start);
   const int item = blockIdx.x;
   if (item >= s_start[E]) return;
   const int e = expert_of_item(s_start, E, item);
   const int64_t r0 = off[e] + static_cast<int64_t>(item - s_start[e]) * kRbRows;
   const int nrows = static_cast<int>(min(off[e + 1] - r0, static_cast<int64_t>(kRbRows)));
-  for (int i = threadIdx.x; i < nrows; i += blockDim.x)
-    s_dz[i] = dz[static_cast<int64_t>(por[r0 + i] / k) * E + e];
+  for (int i = threadIdx.x; i < nrows; i += blockDim.x) {
+    const int t = por[r0 + i] / k;
+    s_dz[i] = dz[static_cast<int64_t>(t) * E + e];
+    if (GATHER) s_tok[i] = t;
+  }
   __syncthreads();
   const int c = (blockIdx.y * kRbThreads + threadIdx.x) * VE;
   if (c < d) {
     float acc[VE];
 #pragma unroll
     for (int q = 0; q < VE; ++q) acc[q] = 0.0f;
-    const T* src = xp + r0 * d + c;
+    const T* src = xp + (GATHER ? 0 : r0 * d) + c;
 #pragma unroll 4
     for (int i = 0; i < nrows; ++i) {
-      const Vec16<T> v = ld16_stream(src + static_cast<int64_t>(i) * d);
+      const int64_t row = GATHER ? static_cast<int64_t>(s_tok[i]) : static_cast<int64_t>(i);
+      const Vec16<T> v = ld16_stream(src + row * d);
       const float g = s_dz[i];
 #pragma unroll
       for (int q = 0; q < VE; ++q) acc[q] = __fmaf_rn(g, v.get(q), acc[q]);
@@ -426,19 +433,30 @@ __global__ void __launch_bounds__(256) router_wgrad_reduce_kernel(
   }
 }
 
+template <typename T>
+static void launch_router_partial(bool gather, dim3 grid, const void* src, const float* dz,
+                                  const int32_t* por, const int64_t* off, int E, int d, int k,
+                                  float* partial, float* partial_db, cudaStream_t s) {
+  if (gather)
+    router_wgrad_partial_kernel<T, true><<<grid, kRbThreads, 0, s>>>(
+        static_cast<const T*>(src), dz, por, off, E, d, k, partial, partial_db);
+  else
+    router_wgrad_partial_kernel<T, false><<<grid, kRbThreads, 0, s>>>(
+        static_cast<const T*>(src), dz, por, off, E, d, k, partial, partial_db);
+}
+
 cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* por,
                               const int64_t* off, int dtype, int64_t rows, int d, int E, int k,
-                              float* dWr, float* db, int accumulate, float* partial, cudaStream_t s) {
+                              float* dWr, float* db, int accumulate, float* partial, cudaStream_t s,
+                              bool gather) {
   const int items = router_bwd_max_items(rows, E);
   float* partial_db = partial + static_cast<int64_t>(items) * d;
   const int vec = dtype == MOE_BF16 ? 8 : 4;
   dim3 grid(items, (d + kRbThreads * vec - 1) / (kRbThreads * vec));
   if (dtype == MOE_BF16)
-    router_wgrad_partial_kernel<bf16><<<grid, kRbThreads, 0, s>>>(
-        static_cast<const bf16*>(xp), dz, por, off, E, d, k, partial, partial_db);
+    launch_router_partial<bf16>(gather, grid, xp, dz, por, off, E, d, k, partial, partial_db, s);
   else
-    router_wgrad_partial_kernel<float><<<grid, kRbThreads, 0, s>>>(
-        static_cast<const float*>(xp), dz, por, off, E, d, k, partial, partial_db);
+    launch_router_partial<float>(gather, grid, xp, dz, por, off, E, d, k, partial, partial_db, s);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(E) * d;

@@ -72,6 +72,15 @@ struct Params {
   float* w2;
   unsigned* err;
   int accumulate;  // wgrad: 1 adds to dW, 0 writes it (zero tiles for experts with no rows)
+  // Gathered A rows (kernels instantiated with GATHER): dispatch row r of the
+  // expert input is row grow[r] / gk of x [gT, d], the token whose copy xp[r]
+  // would be; rows at or past `grows` (the tile's rows past the last expert)
+  // read token 0 and are discarded like any row past the expert's end. Every
+  // gathered box lies inside x: tokens are clamped to [0, gT).
+  const int32_t* grow;
+  int gk;
+  int grows;
+  int gT;
 };
 
 // PAIR: a cluster of two CTAs computes a 256-row tile with one
@@ -240,16 +249,17 @@ __device__ __forceinline__ void issue_loads(const Maps& m, const TileInfo& ti, i
 
 // The same k block for one CTA of a pair: this CTA's 128 rows of A and its
 // half of B (gate/up: CTA 0 stages the Wg rows, CTA 1 the Wu rows), counted
-// on the even CTA's mbarrier at `bar`, a shared::cluster address.
+// on the even CTA's mbarrier at `bar`, a shared::cluster address. With
+// load_a false the A operand is left to the gathered loads.
 template <int KIND, int BN>
 __device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& ti, int kb, int d,
                                                  int f, int cta, uint8_t* a_dst, uint8_t* b_dst,
-                                                 uint32_t bar) {
+                                                 uint32_t bar, bool load_a = true) {
   const int k0 = kb * BK;
   const int arow = ti.row0 + BM * cta;
   constexpr int HALF = BN / 2;
   if (KIND == kFwdGateUp) {
-    tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
+    if (load_a) tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
     tma_load_2d_pair(b_dst, cta == 0 ? &m.b0 : &m.b1, bar, k0, ti.e * f + ti.n0);
   } else if (KIND == kFwdDown) {
     tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
@@ -273,11 +283,47 @@ __device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& 
     const CUtensorMap* bm = ti.prod == 0 ? &m.b0 : (ti.prod == 1 ? &m.b1 : &m.b2);
     const int r = ti.row0 + k0;
     const int mm = ti.m0 + BM * cta;
-    tma_load_2d_pair(a_dst, am, bar, mm, r);
-    tma_load_2d_pair(a_dst + 8192, am, bar, mm + 64, r);
+    if (load_a) {
+      tma_load_2d_pair(a_dst, am, bar, mm, r);
+      tma_load_2d_pair(a_dst + 8192, am, bar, mm + 64, r);
+    }
 #pragma unroll
     for (int j = 0; j < HALF / 64; ++j)
       tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, r);
+  }
+}
+
+// Tokens of the four dispatch rows r0 .. r0 + 3 (one gather4 load).
+__device__ __forceinline__ void gather_tokens(const Params& p, int r0, int (&t)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int r = r0 + q;
+    const int v = r < p.grows ? __ldg(p.grow + r) / p.gk : 0;
+    t[q] = min(max(v, 0), p.gT - 1);
+  }
+}
+
+// Gathered A operand of one pipeline stage, issued by every lane of the
+// producer warp (one tile::gather4 each, four rows of 64 bf16 = 512 bytes).
+// gate/up: lane l stages rows 4l .. 4l+3 of this CTA's 128 rows at K column
+// k0. wgrad (dWg, dWu): A is x^T, K-rows by M-columns; lane l stages the K
+// rows 4 (l % 16) .. +3 of the block for the 64 M columns of box l / 16. The
+// shared-memory image equals that of the tiled load it replaces: the 128-byte
+// swizzle is a function of the destination address and every destination is
+// a 512-byte step from the 1024-aligned stage.
+template <int KIND>
+__device__ __forceinline__ void issue_gather_a(const Maps& m, const TileInfo& ti, int kb, int d,
+                                               int cta, int lane, uint8_t* a_dst, uint32_t bar,
+                                               const int (&t)[4]) {
+  if (KIND == kFwdGateUp) {
+    tma_gather4_pair(a_dst + 512 * lane, &m.a0, bar, kb * BK, t[0], t[1], t[2], t[3]);
+  } else {
+    // columns past d (the last M tile when d is not a multiple of 256) feed
+    // only accumulator rows the epilogue drops: read column 0 there instead
+    const int box = lane >> 4;
+    const int c = ti.m0 + BM * cta + 64 * box;
+    tma_gather4_pair(a_dst + box * 8192 + 512 * (lane & 15), &m.a0, bar, c < d ? c : 0, t[0], t[1],
+                     t[2], t[3]);
   }
 }
 
@@ -554,10 +600,12 @@ __device__ __forceinline__ void issue_mma(uint32_t dtm, uint32_t a_addr, uint32_
   else mma_bf16(dtm, adesc, bdesc, Tr::IDESC, accumulate);
 }
 
-template <int KIND, int BN, bool PAIR>
+template <int KIND, int BN, bool PAIR, bool GATHER>
 __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
   using Tr = Traits<KIND, BN, PAIR>;
+  static_assert(!GATHER || (PAIR && (KIND == kFwdGateUp || KIND == kWgrad)),
+                "gathered A rows: the paired gate/up and weight-gradient kernels");
   constexpr int STAGES = Tr::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -681,6 +729,14 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step) {
       const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
+      // gathered A: this lane's four token rows (gate/up: the same for all k
+      // blocks of the tile; wgrad: those of the next k block, read one block
+      // ahead so the loads' latency hides behind the stage wait)
+      const bool gath = GATHER && (KIND == kFwdGateUp || ti.prod != 2);
+      int tok[4] = {0, 0, 0, 0};
+      if (gath)
+        gather_tokens(p, KIND == kFwdGateUp ? ti.row0 + BM * cta + 4 * lane : ti.row0 + 4 * (lane & 15),
+                      tok);
       for (int kb = 0; kb < nk; ++kb) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, kWaitLimit)) break;
         uint8_t* a_dst = sA + stage * Tr::A_BYTES;
@@ -689,10 +745,15 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         if (lane == 0) {
           if (leader) mbar_arrive_expect_tx(&full[stage], Tr::STAGE_TX);
           if (PAIR) {
-            issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst, full_addr);
+            issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst, full_addr, !gath);
           } else {
             issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
           }
+        }
+        if (GATHER && gath) {
+          issue_gather_a<KIND>(maps, ti, kb, d, cta, lane, a_dst, full_addr, tok);
+          if (KIND == kWgrad && kb + 1 < nk)
+            gather_tokens(p, ti.row0 + (kb + 1) * BK + 4 * (lane & 15), tok);
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -915,11 +976,11 @@ static int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int KIND, int BN, bool PAIR>
+template <int KIND, int BN, bool PAIR, bool GATHER = false>
 static cudaError_t launch(const Maps& m, const Params& p, cudaStream_t s) {
   using Tr = Traits<KIND, BN, PAIR>;
   static_assert(Tr::smem_bytes(kMaxE) <= 232448, "shared memory of one CTA");
-  auto kern = grouped_gemm_kernel<KIND, BN, PAIR>;
+  auto kern = grouped_gemm_kernel<KIND, BN, PAIR, GATHER>;
   const size_t smem = Tr::smem_bytes(p.E);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -970,9 +1031,16 @@ cudaError_t launch_ffn_gateup_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   p.f = a.f;
   p.err = a.err;
   Maps m1{};
-  if (!make_map(&m1.a0, a.xp, d, rows, d, 64, 128) || !make_map(&m1.b0, a.Wg, d, E * f, d, 64, 128) ||
-      !make_map(&m1.b1, a.Wu, d, E * f, d, 64, 128))
+  const bool gather = a.gather.rows != nullptr;
+  // gathered: x [T, d] read four one-row boxes at a time by token index
+  if (!(gather ? make_map(&m1.a0, a.xp, d, static_cast<uint64_t>(a.gather.T), d, 64, 1)
+               : make_map(&m1.a0, a.xp, d, rows, d, 64, 128)) ||
+      !make_map(&m1.b0, a.Wg, d, E * f, d, 64, 128) || !make_map(&m1.b1, a.Wu, d, E * f, d, 64, 128))
     return cudaErrorInvalidValue;
+  p.grow = a.gather.rows;
+  p.gk = a.gather.k;
+  p.grows = static_cast<int>(a.rows);
+  p.gT = static_cast<int>(a.gather.T);
   p.o0 = static_cast<bf16*>(a.h1);
   p.o1 = static_cast<bf16*>(a.h2);
   p.o2 = static_cast<bf16*>(a.a);
@@ -980,7 +1048,7 @@ cudaError_t launch_ffn_gateup_bf16(const FfnFwdArgs& a, cudaStream_t s) {
       (a.h2 && !make_store_map(&m1.o1, a.h2, f, rows)) ||
       (a.a && !make_store_map(&m1.o2, a.a, f, rows)))
     return cudaErrorInvalidValue;
-  return launch<kFwdGateUp, 256, true>(m1, p, s);
+  return gather ? launch<kFwdGateUp, 256, true, true>(m1, p, s) : launch<kFwdGateUp, 256, true>(m1, p, s);
 }
 
 cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
@@ -1052,7 +1120,10 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   const uint64_t rows = static_cast<uint64_t>(a.rows), d = a.d, f = a.f;
   Params p = bwd_params(a);
   Maps m3{};
-  if (!make_map(&m3.a0, a.xp, d, rows, d, 64, 64) || !make_map(&m3.a1, a.a, f, rows, f, 64, 64) ||
+  const bool gather = a.gather.rows != nullptr;
+  if (!(gather ? make_map(&m3.a0, a.xp, d, static_cast<uint64_t>(a.gather.T), d, 64, 1)
+               : make_map(&m3.a0, a.xp, d, rows, d, 64, 64)) ||
+      !make_map(&m3.a1, a.a, f, rows, f, 64, 64) ||
       !make_map(&m3.b0, a.dh1, f, rows, f, 64, 64) || !make_map(&m3.b1, a.dh2, f, rows, f, 64, 64) ||
       !make_map(&m3.b2, a.dyp, d, rows, d, 64, 64))
     return cudaErrorInvalidValue;
@@ -1060,9 +1131,13 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.w1 = a.dWu;
   p.w2 = a.dWd;
   p.accumulate = a.accumulate;
+  p.grow = a.gather.rows;
+  p.gk = a.gather.k;
+  p.grows = static_cast<int>(a.rows);
+  p.gT = static_cast<int>(a.gather.T);
   // CTA pairs: six stages of 32 KB per CTA hide more load latency than four
   // of 48 KB
-  return launch<kWgrad, 256, true>(m3, p, s);
+  return gather ? launch<kWgrad, 256, true, true>(m3, p, s) : launch<kWgrad, 256, true>(m3, p, s);
 }
 
 }  // namespace moe

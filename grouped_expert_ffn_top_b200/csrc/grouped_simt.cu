@@ -19,17 +19,24 @@ __device__ __forceinline__ int expert_of_row(const int64_t* __restrict__ off, in
   return lo;
 }
 
+// Row of the expert input that dispatch row r reads: r itself, or with a
+// gather map the token x[gather_rows[r] / k] that xp[r] copies.
+__device__ __forceinline__ int64_t input_row(const int32_t* __restrict__ grows, int gk, int64_t r) {
+  return grows ? static_cast<int64_t>(grows[r] / gk) : r;
+}
+
 // h1 = xp Wg_e^T, h2 = xp Wu_e^T, a = silu(h1) h2     (one thread per (r, j))
 __global__ void simt_gateup_kernel(const float* __restrict__ xp, const float* __restrict__ Wg,
                                    const float* __restrict__ Wu, const int64_t* __restrict__ off,
                                    int64_t rows, int E, int d, int f, float* __restrict__ h1,
-                                   float* __restrict__ h2, float* __restrict__ a) {
+                                   float* __restrict__ h2, float* __restrict__ a,
+                                   const int32_t* __restrict__ grows, int gk) {
   const int64_t id = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (id >= rows * f) return;
   const int64_t r = id / f;
   const int j = static_cast<int>(id % f);
   const int e = expert_of_row(off, E, r);
-  const float* x = xp + r * d;
+  const float* x = xp + input_row(grows, gk, r) * d;
   const float* g = Wg + (static_cast<int64_t>(e) * f + j) * d;
   const float* u = Wu + (static_cast<int64_t>(e) * f + j) * d;
   float s1 = 0.0f, s2 = 0.0f;
@@ -108,7 +115,8 @@ __global__ void simt_wgrad_kernel(const float* __restrict__ xp, const float* __r
                                   const float* __restrict__ a, const float* __restrict__ dh1,
                                   const float* __restrict__ dh2, const int64_t* __restrict__ off,
                                   int E, int d, int f, float* __restrict__ dWg,
-                                  float* __restrict__ dWu, float* __restrict__ dWd, int accumulate) {
+                                  float* __restrict__ dWu, float* __restrict__ dWd, int accumulate,
+                                  const int32_t* __restrict__ grows, int gk) {
   const int64_t id = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int64_t per = static_cast<int64_t>(f) * d;
   if (id >= E * per) return;
@@ -119,7 +127,7 @@ __global__ void simt_wgrad_kernel(const float* __restrict__ xp, const float* __r
   const int i = static_cast<int>(id % d);
   float sg = 0.0f, su = 0.0f, sd = 0.0f;
   for (int64_t r = r0; r < r1; ++r) {
-    const float xv = xp[r * d + i];
+    const float xv = xp[input_row(grows, gk, r) * d + i];
     sg = __fmaf_rn(dh1[r * f + j], xv, sg);
     su = __fmaf_rn(dh2[r * f + j], xv, su);
   }
@@ -139,7 +147,8 @@ cudaError_t launch_ffn_gateup_f32(const FfnFwdArgs& x, cudaStream_t s) {
   simt_gateup_kernel<<<blocks_for(x.rows * x.f), 256, 0, s>>>(
       static_cast<const float*>(x.xp), static_cast<const float*>(x.Wg),
       static_cast<const float*>(x.Wu), x.offsets, x.rows, x.E, x.d, x.f,
-      static_cast<float*>(x.h1), static_cast<float*>(x.h2), static_cast<float*>(x.a));
+      static_cast<float*>(x.h1), static_cast<float*>(x.h2), static_cast<float*>(x.a),
+      x.gather.rows, x.gather.k);
   return cudaGetLastError();
 }
 
@@ -148,7 +157,8 @@ cudaError_t launch_ffn_fwd_f32(const FfnFwdArgs& x, cudaStream_t s) {
   float* a = static_cast<float*>(x.a);
   simt_gateup_kernel<<<blocks_for(x.rows * x.f), 256, 0, s>>>(
       xp, static_cast<const float*>(x.Wg), static_cast<const float*>(x.Wu), x.offsets, x.rows,
-      x.E, x.d, x.f, static_cast<float*>(x.h1), static_cast<float*>(x.h2), a);
+      x.E, x.d, x.f, static_cast<float*>(x.h1), static_cast<float*>(x.h2), a, x.gather.rows,
+      x.gather.k);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   simt_down_kernel<<<blocks_for(x.rows * x.d), 256, 0, s>>>(
@@ -178,7 +188,7 @@ cudaError_t launch_ffn_wgrad_f32(const FfnBwdArgs& x, cudaStream_t s) {
   simt_wgrad_kernel<<<blocks_for(static_cast<int64_t>(x.E) * x.f * x.d), 256, 0, s>>>(
       static_cast<const float*>(x.xp), static_cast<const float*>(x.dyp),
       static_cast<const float*>(x.a), dh1, dh2, x.offsets, x.E, x.d, x.f, x.dWg, x.dWu, x.dWd,
-      x.accumulate);
+      x.accumulate, x.gather.rows, x.gather.k);
   return cudaGetLastError();
 }
 

@@ -39,11 +39,21 @@ cudaError_t launch_permute_bwd(const void* dxp, const int32_t* row_of_pair, cons
                                const void* Wr, const int32_t* idx, int dtype, int64_t T, int d,
                                int E, int k, void* dX, cudaStream_t s);
 int router_bwd_max_items(int64_t rows, int E);
+// gather: `xp` is x [T, d] and dispatch row r is read as x[pair_of_row[r] / k]
 cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* pair_of_row,
                               const int64_t* offsets, int dtype, int64_t rows, int d, int E, int k,
-                              float* dWr, float* db, int accumulate, float* partial, cudaStream_t s);
+                              float* dWr, float* db, int accumulate, float* partial, cudaStream_t s,
+                              bool gather = false);
 
 // grouped expert FFN (grouped_gemm_sm100.cu, grouped_simt.cu)
+// Gathered dispatch rows: with gather_rows set, `xp` points at x [gather_T, d]
+// and dispatch row r of the expert input is x[gather_rows[r] / gather_k]
+// (gather_rows = pair_of_row), read in place instead of from a permuted copy.
+struct RowGather {
+  const int32_t* rows = nullptr;
+  int k = 1;
+  int64_t T = 0;
+};
 struct FfnFwdArgs {
   const void *xp, *Wg, *Wu, *Wd;
   const int64_t* offsets;
@@ -51,6 +61,7 @@ struct FfnFwdArgs {
   int E, d, f;
   void *h1, *h2, *a, *yp;
   unsigned* err;
+  RowGather gather;
 };
 struct FfnBwdArgs {
   const void *xp, *Wg, *Wu, *Wd, *h1, *h2, *a, *dyp;
@@ -62,6 +73,7 @@ struct FfnBwdArgs {
   void *dh1, *dh2;  // [rows, f]: written by dgrad, read by wgrad
   unsigned* err;
   int accumulate;   // wgrad: 1 adds to dW, 0 writes dW (zero for experts with no rows)
+  RowGather gather; // wgrad: xp's rows gathered from x
 };
 
 cudaError_t launch_selftest_wait_timeout(unsigned* err, long long limit, cudaStream_t s);

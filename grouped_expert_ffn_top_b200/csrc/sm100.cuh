@@ -218,6 +218,20 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 
 // TMA load into this CTA's shared memory whose completion is counted on the
 // mbarrier at `bar_cluster_addr`, which may live in the peer CTA of the pair.
+// TMA gather of four rows: rows r0..r3 of a 2D tensor, columns c0 .. c0 + box
+// width, into four consecutive rows of `dst` (the tensor map's box is one row
+// high). A pair's load counts on the even CTA's barrier at `bar_cluster_addr`.
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int c0, int r0, int r1,
+                                                 int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
+      ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(r0), "r"(r1),
+      "r"(r2), "r"(r3)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
                                                  uint32_t bar_cluster_addr, int c0, int c1) {
   asm volatile(

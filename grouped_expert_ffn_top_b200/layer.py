@@ -9,6 +9,11 @@ With checkpoint=True the forward does not store h1 and h2 and the backward
 first rebuilds them with moe_grouped_ffn_recompute (activation checkpointing:
 2 T k f activation elements less to keep between forward and backward, for
 one more gate/up GEMM).
+With fused_dispatch=True there is no permuted copy xp: the gate/up GEMM, the
+weight gradient's dWg / dWu operand and the router backward read dispatch
+row r in place as x[pair_of_row[r] / k] (moe_grouped_ffn_fwd_gather,
+moe_grouped_ffn_wgrad_gather, moe_router_bwd_gather), with results bitwise
+those of the permuted path; x must then stay unchanged until the backward.
 With a balance-loss coefficient (aux_coef > 0) the forward also calls
 moe_aux_loss after routing, and the backward ends with moe_aux_loss_bwd ->
 moe_router_bwd_dense (the loss's dense logit gradient into dX, dWr, db).
@@ -37,13 +42,15 @@ LAUNCHES_PER_CALL = {
     "router_logits": 1, "route": 3, "permute": 1, "grouped_ffn_fwd": 2, "unpermute_combine": 1,
     "unpermute_combine_bwd": 1, "route_bwd": 1, "grouped_ffn_dgrad": 2, "grouped_ffn_wgrad": 1,
     "permute_bwd": 1, "router_bwd": 2, "aux_loss": 2, "aux_loss_bwd": 1, "router_bwd_dense": 3,
-    "grouped_ffn_recompute": 1,
+    "grouped_ffn_recompute": 1, "grouped_ffn_fwd_gather": 2, "grouped_ffn_wgrad_gather": 1,
+    "router_bwd_gather": 2, "grouped_ffn_recompute_gather": 1,
 }
 
 
 class MoELayer:
     def __init__(self, params: Dict[str, torch.Tensor], k: int, ep_groups: int = 1,
-                 max_tokens: int = 0, aux_coef: float = 0.0, checkpoint: bool = False):
+                 max_tokens: int = 0, aux_coef: float = 0.0, checkpoint: bool = False,
+                 fused_dispatch: bool = False):
         self.Wr, self.b = params["Wr"], params["b"]
         self.Wg, self.Wu, self.Wd = params["Wg"], params["Wu"], params["Wd"]
         self.E, self.f, self.d = self.Wg.shape
@@ -64,6 +71,7 @@ class MoELayer:
         # forward, self.aux holds its loss [1], importance [E], entropy [1]
         self.aux_coef = float(aux_coef)
         self.checkpoint = bool(checkpoint)
+        self.fused = bool(fused_dispatch)
         self.aux = {
             "loss": torch.zeros(1, dtype=f32, device=dev),
             "importance": torch.zeros(self.E, dtype=f32, device=dev),
@@ -82,7 +90,7 @@ class MoELayer:
         f32 = torch.float32
         self.buf = {
             "logits": torch.empty((T, E), dtype=f32, device=dev),
-            "xp": torch.empty((P, d), dtype=dt, device=dev),
+            "xp": torch.empty((0 if self.fused else P, d), dtype=dt, device=dev),
             "h1": torch.empty((P, f), dtype=dt, device=dev),
             "h2": torch.empty((P, f), dtype=dt, device=dev),
             "a": torch.empty((P, f), dtype=dt, device=dev),
@@ -145,14 +153,19 @@ class MoELayer:
             N.moe_aux_loss(v["logits"], r["counts"], self.k, self.aux_coef, self.aux, self.ws["aux"],
                            stream)
             mark("aux_loss")
-        N.moe_permute(x, r["row_of_pair"], self.k, v["xp"], stream)
-        mark("permute")
         saved = {n: v[n] for n in ("h1", "h2", "a", "yp")}
         if self.checkpoint:
             saved["h1"] = saved["h2"] = None  # rebuilt in the backward
-        N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"], saved, self.ws["ffn_fwd"],
-                              stream)
-        mark("grouped_ffn_fwd")
+        if self.fused:
+            N.moe_grouped_ffn_fwd_gather(x, r["pair_of_row"], self.k, self.Wg, self.Wu, self.Wd, r["offsets"],
+                                         saved, self.ws["ffn_fwd"], stream)
+            mark("grouped_ffn_fwd_gather")
+        else:
+            N.moe_permute(x, r["row_of_pair"], self.k, v["xp"], stream)
+            mark("permute")
+            N.moe_grouped_ffn_fwd(v["xp"], self.Wg, self.Wu, self.Wd, r["offsets"], saved, self.ws["ffn_fwd"],
+                                  stream)
+            mark("grouped_ffn_fwd")
         Y = v["Y"] if out is None else out
         N.moe_unpermute_combine(v["yp"], r["topk_w"], r["row_of_pair"], Y, stream)
         mark("unpermute_combine")
@@ -172,23 +185,38 @@ class MoELayer:
         mark("unpermute_combine_bwd")
         N.moe_route_bwd(v["dg"], r["topk_w"], r["topk_idx"], self.E, v["dlogits"], stream)
         mark("route_bwd")
-        if self.checkpoint:
+        if self.checkpoint and self.fused:
+            N.moe_grouped_ffn_recompute_gather(self.x, r["pair_of_row"], self.k, self.Wg, self.Wu, r["offsets"],
+                                               v["h1"], v["h2"], self.ws["ffn_bwd"], stream)
+            mark("grouped_ffn_recompute_gather")
+        elif self.checkpoint:
             N.moe_grouped_ffn_recompute(v["xp"], self.Wg, self.Wu, r["offsets"], v["h1"], v["h2"],
                                         self.ws["ffn_bwd"], stream)
             mark("grouped_ffn_recompute")
         N.moe_grouped_ffn_dgrad(self.Wg, self.Wu, self.Wd, v["h1"], v["h2"], v["dyp"], r["offsets"],
                                 v["dh1"], v["dh2"], v["dxp"], self.ws["ffn_bwd"], stream)
         mark("grouped_ffn_dgrad")
-        N.moe_grouped_ffn_wgrad(v["xp"], v["a"], v["dyp"], v["dh1"], v["dh2"], r["offsets"], g["dWg"],
-                                g["dWu"], g["dWd"], self.ws["ffn_bwd"], stream, accumulate=accumulate)
-        mark("grouped_ffn_wgrad")
+        if self.fused:
+            N.moe_grouped_ffn_wgrad_gather(self.x, r["pair_of_row"], self.k, v["a"], v["dyp"], v["dh1"], v["dh2"],
+                                           r["offsets"], g["dWg"], g["dWu"], g["dWd"], self.ws["ffn_bwd"],
+                                           stream, accumulate=accumulate)
+            mark("grouped_ffn_wgrad_gather")
+        else:
+            N.moe_grouped_ffn_wgrad(v["xp"], v["a"], v["dyp"], v["dh1"], v["dh2"], r["offsets"], g["dWg"],
+                                    g["dWu"], g["dWd"], self.ws["ffn_bwd"], stream, accumulate=accumulate)
+            mark("grouped_ffn_wgrad")
         dX = v["dX"] if out is None else out
         N.moe_permute_bwd(v["dxp"], r["row_of_pair"], v["dlogits"], self.Wr, r["topk_idx"], T, self.k,
                           dX, stream)
         mark("permute_bwd")
-        N.moe_router_bwd(v["xp"], v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"], g["db"],
-                         self.ws["router_bwd"], stream, accumulate=accumulate)
-        mark("router_bwd")
+        if self.fused:
+            N.moe_router_bwd_gather(self.x, v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"],
+                                    g["db"], self.ws["router_bwd"], stream, accumulate=accumulate)
+            mark("router_bwd_gather")
+        else:
+            N.moe_router_bwd(v["xp"], v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"], g["db"],
+                             self.ws["router_bwd"], stream, accumulate=accumulate)
+            mark("router_bwd")
         if self.aux_coef:
             N.moe_aux_loss_bwd(v["logits"], r["counts"], self.k, self.aux_coef, aux_dloss, v["dz_aux"],
                                stream)

@@ -73,6 +73,15 @@ _SIGNATURES = {
     "moe_aux_loss_bwd": ([_p, _p, _i64, _i, _i, _f, _f, _p, _p], _i),
     "moe_router_bwd_dense_workspace_bytes": ([_i64, _i, _i], _sz),
     "moe_router_bwd_dense": ([_p, _p, _p, _i, _i64, _i, _i, _p, _p, _p, _i, _p, _sz, _p], _i),
+    "moe_grouped_ffn_fwd_gather": ([_p, _p, _i64, _i, _p, _p, _p, _i, _p, _i, _i, _i, _p, _p, _p, _p, _p, _sz,
+                                    _p], _i),
+    "moe_grouped_ffn_recompute_gather": ([_p, _p, _i64, _i, _p, _p, _i, _p, _i, _i, _i, _p, _p, _p, _sz, _p],
+                                         _i),
+    "moe_grouped_ffn_bwd_gather": ([_p, _p, _i64, _i] + [_p] * 7 + [_i, _p, _i, _i, _i, _p, _p, _p, _p, _i, _p,
+                                                                   _sz, _p], _i),
+    "moe_grouped_ffn_wgrad_gather": ([_p, _p, _i64, _i] + [_p] * 4 + [_i, _p, _i, _i, _i, _p, _p, _p, _i, _p,
+                                                                     _sz, _p], _i),
+    "moe_router_bwd_gather": ([_p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p, _i, _p, _sz, _p], _i),
 }
 
 
@@ -229,6 +238,40 @@ def moe_grouped_ffn_recompute(xp, Wg, Wu, expert_offsets, h1, h2, ws=None, strea
            "moe_grouped_ffn_recompute")
 
 
+def moe_grouped_ffn_fwd_gather(x, pair_of_row, k: int, Wg, Wu, Wd, expert_offsets, out=None, ws=None,
+                               stream=None):
+    """moe_grouped_ffn_fwd on the dispatch rows x[pair_of_row[r] // k], read
+    in place (no permuted copy)."""
+    _contig(x, pair_of_row, Wg, Wu, Wd, expert_offsets)
+    T, d = x.shape
+    E, f, _ = Wg.shape
+    rows, dt = T * k, _dt(x)
+    if out is None:
+        out = {n: torch.empty((rows, f), dtype=x.dtype, device=x.device) for n in ("h1", "h2", "a")}
+        out["yp"] = torch.empty((rows, d), dtype=x.dtype, device=x.device)
+    if ws is None:
+        ws = _ws(moe_grouped_ffn_fwd_workspace_bytes(rows, E, d, f, dt), x.device)
+    _check(lib().moe_grouped_ffn_fwd_gather(_ptr(x), _ptr(pair_of_row), T, k, _ptr(Wg), _ptr(Wu), _ptr(Wd), dt,
+                                            _ptr(expert_offsets), E, d, f, _ptr(out["h1"]), _ptr(out["h2"]),
+                                            _ptr(out["a"]), _ptr(out["yp"]), _ptr(ws), ws.numel(),
+                                            _stream(stream)), "moe_grouped_ffn_fwd_gather")
+    return out
+
+
+def moe_grouped_ffn_recompute_gather(x, pair_of_row, k: int, Wg, Wu, expert_offsets, h1, h2, ws=None,
+                                     stream=None):
+    _contig(x, pair_of_row, Wg, Wu, expert_offsets, h1, h2)
+    T, d = x.shape
+    E, f, _ = Wg.shape
+    dt = _dt(x)
+    if ws is None:
+        ws = _ws(moe_grouped_ffn_fwd_workspace_bytes(T * k, E, d, f, dt), x.device)
+    _check(lib().moe_grouped_ffn_recompute_gather(_ptr(x), _ptr(pair_of_row), T, k, _ptr(Wg), _ptr(Wu), dt,
+                                                  _ptr(expert_offsets), E, d, f, _ptr(h1), _ptr(h2), _ptr(ws),
+                                                  ws.numel(), _stream(stream)),
+           "moe_grouped_ffn_recompute_gather")
+
+
 def moe_unpermute_combine(yp, topk_w, row_of_pair, Y=None, stream=None):
     _contig(yp, topk_w, row_of_pair)
     T, k = topk_w.shape
@@ -333,6 +376,24 @@ def moe_grouped_ffn_bwd(xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu
     return dxp
 
 
+def moe_grouped_ffn_bwd_gather(x, pair_of_row, k: int, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu,
+                               dWd, dxp=None, ws=None, stream=None, accumulate: bool = True):
+    _contig(x, pair_of_row, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu, dWd)
+    T, d = x.shape
+    E, f, _ = Wg.shape
+    rows, dt = T * k, _dt(x)
+    if dxp is None:
+        dxp = torch.empty((rows, d), dtype=x.dtype, device=x.device)
+    if ws is None:
+        ws = _ws(moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dt), x.device)
+    _check(lib().moe_grouped_ffn_bwd_gather(_ptr(x), _ptr(pair_of_row), T, k, _ptr(Wg), _ptr(Wu), _ptr(Wd),
+                                            _ptr(h1), _ptr(h2), _ptr(a), _ptr(dyp), dt, _ptr(expert_offsets),
+                                            E, d, f, _ptr(dxp), _ptr(dWg), _ptr(dWu), _ptr(dWd),
+                                            int(accumulate), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_grouped_ffn_bwd_gather")
+    return dxp
+
+
 def moe_grouped_ffn_dgrad(Wg, Wu, Wd, h1, h2, dyp, expert_offsets, dh1, dh2, dxp, ws, stream=None):
     _contig(Wg, Wu, Wd, h1, h2, dyp, expert_offsets, dh1, dh2, dxp)
     rows, d = dyp.shape
@@ -354,6 +415,18 @@ def moe_grouped_ffn_wgrad(xp, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd, w
                                        _ptr(dWd), int(accumulate), _ptr(ws), ws.numel(),
                                        _stream(stream)),
            "moe_grouped_ffn_wgrad")
+
+
+def moe_grouped_ffn_wgrad_gather(x, pair_of_row, k: int, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd, ws,
+                                 stream=None, accumulate: bool = True):
+    _contig(x, pair_of_row, a, dyp, dh1, dh2, expert_offsets, dWg, dWu, dWd)
+    T, d = x.shape
+    E, f, _ = dWg.shape
+    _check(lib().moe_grouped_ffn_wgrad_gather(_ptr(x), _ptr(pair_of_row), T, k, _ptr(a), _ptr(dyp), _ptr(dh1),
+                                              _ptr(dh2), _dt(x), _ptr(expert_offsets), E, d, f, _ptr(dWg),
+                                              _ptr(dWu), _ptr(dWd), int(accumulate), _ptr(ws), ws.numel(),
+                                              _stream(stream)),
+           "moe_grouped_ffn_wgrad_gather")
 
 
 def moe_permute_bwd(dxp, row_of_pair, dlogits, Wr, topk_idx, T: int, k: int, dX=None, stream=None):
@@ -381,3 +454,16 @@ def moe_router_bwd(xp, dlogits, pair_of_row, expert_offsets, k: int, dWr, db, ws
     _check(lib().moe_router_bwd(_ptr(xp), _ptr(dlogits), _ptr(pair_of_row), _ptr(expert_offsets),
                                 _dt(xp), T, d, E, k, _ptr(dWr), _ptr(db), int(accumulate), _ptr(ws),
                                 ws.numel(), _stream(stream)), "moe_router_bwd")
+
+
+def moe_router_bwd_gather(x, dlogits, pair_of_row, expert_offsets, k: int, dWr, db, ws=None, stream=None,
+                          accumulate: bool = True):
+    """moe_router_bwd reading dispatch row r as x[pair_of_row[r] // k]."""
+    _contig(x, dlogits, pair_of_row, expert_offsets, dWr, db)
+    T, d = x.shape
+    E = dlogits.shape[1]
+    if ws is None:
+        ws = _ws(moe_router_bwd_workspace_bytes(T * k, d, E), x.device)
+    _check(lib().moe_router_bwd_gather(_ptr(x), _ptr(dlogits), _ptr(pair_of_row), _ptr(expert_offsets),
+                                       _dt(x), T, d, E, k, _ptr(dWr), _ptr(db), int(accumulate), _ptr(ws),
+                                       ws.numel(), _stream(stream)), "moe_router_bwd_gather")

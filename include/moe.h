@@ -221,6 +221,22 @@ MOE_API int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, 
                         int d, int f, void* h1, void* h2, void* a, void* yp,
                         void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Fused dispatch (the permute folded into the expert GEMMs' operand loads;
+ * EP token dispatch, leap-finetune PR #26 "Add MoE expert parallel training
+ * runtime", Summary): moe_grouped_ffn_fwd with the expert input read in place
+ * from the tokens instead of from the permuted copy xp. Dispatch row r of the
+ * expert input is x[pair_of_row[r] / k], exactly the row moe_permute copies
+ * to xp[r], so every output is bitwise that of moe_permute followed by
+ * moe_grouped_ffn_fwd; xp is neither written nor read.
+ *   x [T, d] dtype; pair_of_row [T*k] int32 (moe_route's output); rows = T*k;
+ *   every other argument and error as moe_grouped_ffn_fwd (k in 1..32).
+ * The bf16 path loads the rows with TMA tile::gather4 (four rows a load). */
+MOE_API int moe_grouped_ffn_fwd_gather(const void* x, const int32_t* pair_of_row, int64_t T, int k,
+                                       const void* Wg, const void* Wu, const void* Wd, int dtype,
+                                       const int64_t* expert_offsets, int E, int d, int f,
+                                       void* h1, void* h2, void* a, void* yp, void* ws,
+                                       size_t ws_bytes, cudaStream_t stream);
+
 /* Unpermute and weighted combine (full source-order outputs, ART issue
  * #917 Desired behavior):
  *   Y[t, :] = sum_{j<k} topk_w[t,j] * yp[row_of_pair[t*k+j], :]
@@ -257,6 +273,14 @@ MOE_API int moe_grouped_ffn_recompute(const void* xp, const void* Wg, const void
                                       int f, void* h1, void* h2, void* ws, size_t ws_bytes,
                                       cudaStream_t stream);
 
+/* moe_grouped_ffn_recompute with the expert input gathered from x through
+ * pair_of_row (rows = T*k), as moe_grouped_ffn_fwd_gather. */
+MOE_API int moe_grouped_ffn_recompute_gather(const void* x, const int32_t* pair_of_row, int64_t T,
+                                             int k, const void* Wg, const void* Wu, int dtype,
+                                             const int64_t* expert_offsets, int E, int d, int f,
+                                             void* h1, void* h2, void* ws, size_t ws_bytes,
+                                             cudaStream_t stream);
+
 /* Workspace of moe_grouped_ffn_bwd, in bytes (holds dh1 and dh2). */
 MOE_API size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype);
 
@@ -276,6 +300,18 @@ MOE_API int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, 
                         int dtype, const int64_t* expert_offsets, int64_t rows, int E, int d,
                         int f, void* dxp, float* dWg, float* dWu, float* dWd, int accumulate,
                         void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* moe_grouped_ffn_bwd with xp (the weight gradients' dWg, dWu operand) read
+ * in place from x through pair_of_row (rows = T*k), as
+ * moe_grouped_ffn_fwd_gather; bitwise the results of moe_grouped_ffn_bwd on
+ * moe_permute's xp. dxp stays in dispatch-row order. */
+MOE_API int moe_grouped_ffn_bwd_gather(const void* x, const int32_t* pair_of_row, int64_t T, int k,
+                                       const void* Wg, const void* Wu, const void* Wd,
+                                       const void* h1, const void* h2, const void* a,
+                                       const void* dyp, int dtype, const int64_t* expert_offsets,
+                                       int E, int d, int f, void* dxp, float* dWg, float* dWu,
+                                       float* dWd, int accumulate, void* ws, size_t ws_bytes,
+                                       cudaStream_t stream);
 
 /* The two halves of moe_grouped_ffn_bwd, for callers that keep dh1 / dh2
  * themselves (and may schedule the weight gradient apart from the data
@@ -297,6 +333,14 @@ MOE_API int moe_grouped_ffn_wgrad(const void* xp, const void* a, const void* dyp
                                   int64_t rows, int E, int d, int f, float* dWg, float* dWu,
                                   float* dWd, int accumulate, void* ws, size_t ws_bytes,
                                   cudaStream_t stream);
+/* moe_grouped_ffn_wgrad with xp gathered from x through pair_of_row
+ * (rows = T*k), as moe_grouped_ffn_fwd_gather. */
+MOE_API int moe_grouped_ffn_wgrad_gather(const void* x, const int32_t* pair_of_row, int64_t T,
+                                         int k, const void* a, const void* dyp, const void* dh1,
+                                         const void* dh2, int dtype, const int64_t* expert_offsets,
+                                         int E, int d, int f, float* dWg, float* dWu, float* dWd,
+                                         int accumulate, void* ws, size_t ws_bytes,
+                                         cudaStream_t stream);
 
 /* Permute backward, with the router's input gradient folded in:
  *   dX[t, :] = sum_{j<k} dxp[row_of_pair[t*k+j], :]
@@ -334,6 +378,13 @@ MOE_API int moe_router_bwd(const void* xp, const float* dlogits, const int32_t* 
                            const int64_t* expert_offsets, int dtype, int64_t T, int d, int E,
                            int k, float* dWr, float* db, int accumulate, void* ws,
                            size_t ws_bytes, cudaStream_t stream);
+/* moe_router_bwd reading dispatch row r as x[pair_of_row[r] / k] (x [T, d])
+ * instead of xp[r]: the same values in the same order, so bitwise the same
+ * dWr and db, without the permuted copy. */
+MOE_API int moe_router_bwd_gather(const void* x, const float* dlogits, const int32_t* pair_of_row,
+                                  const int64_t* expert_offsets, int dtype, int64_t T, int d,
+                                  int E, int k, float* dWr, float* db, int accumulate, void* ws,
+                                  size_t ws_bytes, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------
  * Auxiliary load-balancing loss of the router and routing metrics.

@@ -137,3 +137,38 @@ def test_balance_loss_argument_errors(L):
     assert L.moe_router_bwd_dense(*args, 2, null, 0, null) == N.MOE_ERR_INVALID_ARG  # accumulate
     assert L.moe_router_bwd_dense(*args, 1, null, 0, null) == N.MOE_ERR_INVALID_ARG  # null dWr
     assert L.moe_router_bwd_dense_workspace_bytes(512, 128, 8) >= 256 + 4 * 2 * 8 * 129
+
+
+def test_gathered_dispatch_argument_errors(L):
+    """The fused-dispatch entries check k, T and the row map before anything
+    else (a fake non-null address stands in for pair_of_row: it is never read
+    because every call here is rejected or has nothing to do)."""
+    fake = ctypes.c_void_p(256)
+    tail = [null] * 4 + [null, 0, null]  # h1, h2, a, yp, ws, ws_bytes, stream
+    fwd = lambda por, T, k, dt=N.MOE_BF16, d=128: L.moe_grouped_ffn_fwd_gather(  # noqa: E731
+        null, por, T, k, null, null, null, dt, null, 4, d, 128, *tail)
+    assert fwd(null, 10, 2) == N.MOE_ERR_INVALID_ARG  # no row map
+    assert b"null pointer" in L.moe_last_error()
+    assert fwd(fake, 10, 0) == N.MOE_ERR_INVALID_ARG  # k < 1
+    assert fwd(fake, 10, 33) == N.MOE_ERR_UNSUPPORTED  # k > 32
+    assert fwd(fake, 10, 2, d=100) == N.MOE_ERR_UNSUPPORTED  # bf16 d % 64
+    assert fwd(fake, -1, 2) == N.MOE_ERR_INVALID_ARG
+    assert fwd(fake, 0, 2) == N.MOE_OK  # no tokens: nothing to do
+    assert fwd(fake, 10, 2) == N.MOE_ERR_INVALID_ARG  # null operands
+    rec = L.moe_grouped_ffn_recompute_gather(null, fake, 10, 0, null, null, N.MOE_BF16, null, 4, 128, 128,
+                                             null, null, null, 0, null)
+    assert rec == N.MOE_ERR_INVALID_ARG
+    wg = lambda acc, T=0: L.moe_grouped_ffn_wgrad_gather(  # noqa: E731
+        null, fake, T, 2, null, null, null, null, N.MOE_BF16, null, 4, 128, 128, null, null, null, acc,
+        null, 0, null)
+    assert wg(1) == N.MOE_OK  # empty batch, adding: nothing to do
+    assert wg(2) == N.MOE_ERR_INVALID_ARG
+    assert wg(0) == N.MOE_ERR_INVALID_ARG  # writing needs dW
+    bw = L.moe_grouped_ffn_bwd_gather(null, null, 5, 2, *([null] * 7), N.MOE_BF16, null, 4, 128, 128,
+                                      *([null] * 4), 1, null, 0, null)
+    assert bw == N.MOE_ERR_INVALID_ARG
+    rb = lambda T, k, acc: L.moe_router_bwd_gather(null, null, fake, null, N.MOE_BF16, T, 128, 8, k,  # noqa: E731
+                                                  null, null, acc, null, 0, null)
+    assert rb(0, 2, 1) == N.MOE_OK
+    assert rb(4, 9, 1) == N.MOE_ERR_INVALID_ARG  # k > E
+    assert rb(4, 2, 1) == N.MOE_ERR_INVALID_ARG  # null operands
