@@ -76,7 +76,8 @@ struct Params {
   // expert input is row grow[r] / gk of x [gT, d], the token whose copy xp[r]
   // would be; rows at or past `grows` (the tile's rows past the last expert)
   // read token 0 and are discarded like any row past the expert's end. Every
-  // gathered box lies inside x: tokens are clamped to [0, gT).
+  // gathered address lies inside x: tokens are clamped to [0, gT).
+  const bf16* gx;
   const int32_t* grow;
   int gk;
   int grows;
@@ -112,7 +113,7 @@ struct Traits {
   // N extent of one output tile (gate/up: 128 f columns, each with its gate
   // and up accumulator, together the MMA's N = 256)
   static constexpr int NTILE = KIND == kFwdGateUp ? 128 : BN;
-  static constexpr size_t BAR_BYTES = 256;
+  static constexpr size_t BAR_BYTES = 320;
   // dynamic shared memory: alignment slack, stages, barriers, and the tile
   // schedule (expert offsets, first tile and expert of each slot) for E experts
   static constexpr size_t SMEM_FIXED =
@@ -293,37 +294,54 @@ __device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& 
   }
 }
 
-// Tokens of the four dispatch rows r0 .. r0 + 3 (one gather4 load).
-__device__ __forceinline__ void gather_tokens(const Params& p, int r0, int (&t)[4]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int r = r0 + q;
-    const int v = r < p.grows ? __ldg(p.grow + r) / p.gk : 0;
-    t[q] = min(max(v, 0), p.gT - 1);
-  }
+// Token of dispatch row r (see Params::grow).
+__device__ __forceinline__ int token_of_row(const Params& p, int r) {
+  const int v = r < p.grows ? __ldg(p.grow + r) / p.gk : 0;
+  return min(max(v, 0), p.gT - 1);
 }
 
-// Gathered A operand of one pipeline stage, issued by every lane of the
-// producer warp (one tile::gather4 each, four rows of 64 bf16 = 512 bytes).
-// gate/up: lane l stages rows 4l .. 4l+3 of this CTA's 128 rows at K column
-// k0. wgrad (dWg, dWu): A is x^T, K-rows by M-columns; lane l stages the K
-// rows 4 (l % 16) .. +3 of the block for the 64 M columns of box l / 16. The
-// shared-memory image equals that of the tiled load it replaces: the 128-byte
-// swizzle is a function of the destination address and every destination is
-// a 512-byte step from the 1024-aligned stage.
+// Gathered A operand of one pipeline stage, written by the 32 lanes of the
+// producer warp with 16-byte cp.async copies into the 128-byte-swizzled
+// layout the tiled TMA load would produce (16-byte chunk c of smem row j goes
+// to chunk c ^ (j % 8); the stage is 1024-byte aligned). Each warp-wide copy
+// moves four 128-byte row segments. Completion is counted on the local
+// mbarrier by the caller's cp.async arrive.
+//   gate/up: smem row j (0..127) = dispatch row row0 + 128 cta + j at K
+//     columns k0 .. k0 + 63; lane l holds in tok[q] the token of row l + 32 q.
+//   wgrad (dWg, dWu; A = x^T, M-major): smem row j (0..63) of box b = K row j
+//     of the block (dispatch row row0 + k0 + j), M columns col0 + 64 b ..;
+//     lane l holds in tok[q] the token of K row l + 32 q. Columns past d (the
+//     last M tile when d is not a multiple of 256) feed only accumulator rows
+//     the epilogue drops: they read column 0 instead.
 template <int KIND>
-__device__ __forceinline__ void issue_gather_a(const Maps& m, const TileInfo& ti, int kb, int d,
-                                               int cta, int lane, uint8_t* a_dst, uint32_t bar,
-                                               const int (&t)[4]) {
+__device__ __forceinline__ void gather_a_stage(const Params& p, int lane, uint32_t a_s, int k0,
+                                               int col0, const int (&tok)[4]) {
+  const char* xb = reinterpret_cast<const char*>(p.gx);
+  const int c = lane & 7;
   if (KIND == kFwdGateUp) {
-    tma_gather4_pair(a_dst + 512 * lane, &m.a0, bar, kb * BK, t[0], t[1], t[2], t[3]);
+    const int h = lane >> 3;  // row 4 i + h of iteration i
+    const uint32_t d_even = h * 128 + ((c ^ h) << 4);        // (4 i + h) % 8 = h for even i
+    const uint32_t d_odd = h * 128 + ((c ^ (h + 4)) << 4);   // and 4 + h for odd i
+    const int64_t cofs = static_cast<int64_t>(k0 + 8 * c) * 2;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int t = __shfl_sync(0xffffffffu, tok[i >> 3], (4 * i + h) & 31);
+      cp_async_16(a_s + i * 512 + ((i & 1) ? d_odd : d_even),
+                  xb + static_cast<int64_t>(t) * p.d * 2 + cofs);
+    }
   } else {
-    // columns past d (the last M tile when d is not a multiple of 256) feed
-    // only accumulator rows the epilogue drops: read column 0 there instead
-    const int box = lane >> 4;
-    const int c = ti.m0 + BM * cta + 64 * box;
-    tma_gather4_pair(a_dst + box * 8192 + 512 * (lane & 15), &m.a0, bar, c < d ? c : 0, t[0], t[1],
-                     t[2], t[3]);
+    const int hh = lane >> 4;        // K row 2 i + hh of iteration i
+    const int b = (lane >> 3) & 1;   // M box
+    int col = col0 + 64 * b + 8 * c;
+    if (col >= p.d) col = 0;
+    const int64_t cofs = static_cast<int64_t>(col) * 2;
+    const uint32_t dbase = b * 8192 + hh * 128;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int t = __shfl_sync(0xffffffffu, tok[i >> 4], (2 * i + hh) & 31);
+      const uint32_t sw = static_cast<uint32_t>(c ^ ((2 * (i & 3) + hh) & 7)) << 4;
+      cp_async_16(a_s + dbase + i * 256 + sw, xb + static_cast<int64_t>(t) * p.d * 2 + cofs);
+    }
   }
 }
 
@@ -600,6 +618,19 @@ __device__ __forceinline__ void issue_mma(uint32_t dtm, uint32_t a_addr, uint32_
   else mma_bf16(dtm, adesc, bdesc, Tr::IDESC, accumulate);
 }
 
+// The MMA issuer's wait for a stage: its TMA loads (and, in a gathered
+// kernel, the odd CTA's relayed rows) on `full`, and this CTA's own gathered
+// rows on `gfull`, made visible to the tensor core's operand reads.
+template <bool GATHER>
+__device__ __forceinline__ bool wait_stage(uint64_t* full, uint64_t* gfull, int stage,
+                                           uint32_t phase, volatile int* abort) {
+  if (GATHER) {
+    if (!wait_bounded(&gfull[stage], phase, abort, kWaitLimit)) return false;
+    fence_proxy_async_all();
+  }
+  return wait_bounded(&full[stage], phase, abort, kWaitLimit);
+}
+
 template <int KIND, int BN, bool PAIR, bool GATHER>
 __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ Maps maps, const Params p) {
@@ -620,7 +651,8 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* lbar = drain + 1;  // [8] SwiGLU-backward epilogue loads: two per epilogue warp
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(lbar + 8);
+  uint64_t* gfull = lbar + 8;  // [STAGES] gathered kernels: this CTA's cp.async rows landed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gfull + STAGES);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort) + 1;
   int64_t* s_off = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(bars) + Tr::BAR_BYTES);
@@ -639,8 +671,11 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // gathered kernels: the even CTA's producer arrival (with the TMA
+      // bytes) and the odd CTA's relay of its gathered rows
+      mbar_init(&full[s], GATHER ? 2 : 1);
       mbar_init(&empty[s], 1);
+      if (GATHER) mbar_init(&gfull[s], 32);  // one cp.async arrival per producer lane
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -729,31 +764,43 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step) {
       const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
-      // gathered A: this lane's four token rows (gate/up: the same for all k
-      // blocks of the tile; wgrad: those of the next k block, read one block
-      // ahead so the loads' latency hides behind the stage wait)
+      // gathered A: the tokens of this lane's rows (gate/up: rows l + 32 q of
+      // the CTA's 128, the same for all k blocks of the tile; wgrad: K rows
+      // l + 32 q of the k block, read one block ahead so that the loads'
+      // latency hides behind the stage wait)
       const bool gath = GATHER && (KIND == kFwdGateUp || ti.prod != 2);
       int tok[4] = {0, 0, 0, 0};
-      if (gath)
-        gather_tokens(p, KIND == kFwdGateUp ? ti.row0 + BM * cta + 4 * lane : ti.row0 + 4 * (lane & 15),
-                      tok);
+      if (gath) {
+        const int r0 = KIND == kFwdGateUp ? ti.row0 + BM * cta : ti.row0;
+#pragma unroll
+        for (int q = 0; q < (KIND == kFwdGateUp ? 4 : 2); ++q) tok[q] = token_of_row(p, r0 + lane + 32 * q);
+      }
+      // the TMA bytes of a stage: without the gathered A rows
+      const uint32_t stage_tx = gath ? Tr::STAGE_TX - (PAIR ? 2 : 1) * Tr::A_BYTES : Tr::STAGE_TX;
       for (int kb = 0; kb < nk; ++kb) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, s_abort, kWaitLimit)) break;
         uint8_t* a_dst = sA + stage * Tr::A_BYTES;
         uint8_t* b_dst = sB + stage * Tr::B_BYTES;
         const uint32_t full_addr = full_leader + 8u * static_cast<uint32_t>(stage);
         if (lane == 0) {
-          if (leader) mbar_arrive_expect_tx(&full[stage], Tr::STAGE_TX);
+          if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
           if (PAIR) {
             issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst, full_addr, !gath);
           } else {
             issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
           }
         }
-        if (GATHER && gath) {
-          issue_gather_a<KIND>(maps, ti, kb, d, cta, lane, a_dst, full_addr, tok);
-          if (KIND == kWgrad && kb + 1 < nk)
-            gather_tokens(p, ti.row0 + (kb + 1) * BK + 4 * (lane & 15), tok);
+        if (GATHER) {
+          if (gath) {
+            gather_a_stage<KIND>(p, lane, smem_u32(a_dst), kb * BK, ti.m0 + BM * cta, tok);
+            if (KIND == kWgrad && kb + 1 < nk) {
+              tok[0] = token_of_row(p, ti.row0 + (kb + 1) * BK + lane);
+              tok[1] = token_of_row(p, ti.row0 + (kb + 1) * BK + lane + 32);
+            }
+          }
+          // every stage of a gathered kernel completes gfull (with no copies
+          // of this stage the arrival waits only for earlier ones)
+          cp_async_mbar_arrive_noinc(&gfull[stage]);
         }
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -763,6 +810,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         }
       }
     }
+    if (GATHER) cp_async_wait_all();
     if (*s_abort) {
       // leave no copy in flight into shared memory that is about to be freed
       // (a pair's loads all count on the even CTA's barriers)
@@ -790,7 +838,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       // pipe idle between instructions).
       const int nfull = KIND == kWgrad ? ti.rows / BK : nk;
       for (int kb = 0; kb < nfull; ++kb) {
-        if (!wait_bounded(&full[stage], phase, s_abort, kWaitLimit)) {
+        if (!wait_stage<GATHER>(full, gfull, stage, phase, s_abort)) {
           ok = false;
           break;
         }
@@ -817,7 +865,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         // hold valid rows run, and the invalid rows inside the last of them
         // are zeroed in both operands first.
         const int kb = nfull;
-        if (!wait_bounded(&full[stage], phase, s_abort, kWaitLimit)) {
+        if (!wait_stage<GATHER>(full, gfull, stage, phase, s_abort)) {
           ok = false;
         } else {
           tc_fence_after();
@@ -874,6 +922,32 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     __syncwarp();
     volatile int never = 0;
     wait_bounded(drain, 0, &never, kWaitLimit);
+  } else if (GATHER && warp == 1) {
+    // --------------------------------- odd CTA: relay of its gathered rows
+    // The even CTA's MMA reads this CTA's A stage too; once this CTA's
+    // cp.async rows of a stage have landed, pass that on to the even CTA's
+    // full barrier (in the producer's stage order).
+    int stage = 0;
+    uint32_t phase = 0;
+    const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+    bool ok = true;
+    for (int tile = first_tile; ok && tile < total && !*s_abort; tile += tile_step) {
+      const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
+      const int nk = num_kblocks<KIND, BN>(ti, d, f);
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bounded(&gfull[stage], phase, s_abort, kWaitLimit)) {
+          ok = false;
+          break;
+        }
+        fence_proxy_async_all();
+        if (lane == 0) mbar_arrive_cluster(full_leader + 8u * static_cast<uint32_t>(stage));
+        __syncwarp();
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
   } else if (warp >= 2) {
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;
@@ -1032,11 +1106,12 @@ cudaError_t launch_ffn_gateup_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   p.err = a.err;
   Maps m1{};
   const bool gather = a.gather.rows != nullptr;
-  // gathered: x [T, d] read four one-row boxes at a time by token index
+  // gathered: the kernel reads x [T, d] itself (the map stays valid but unused)
   if (!(gather ? make_map(&m1.a0, a.xp, d, static_cast<uint64_t>(a.gather.T), d, 64, 1)
                : make_map(&m1.a0, a.xp, d, rows, d, 64, 128)) ||
       !make_map(&m1.b0, a.Wg, d, E * f, d, 64, 128) || !make_map(&m1.b1, a.Wu, d, E * f, d, 64, 128))
     return cudaErrorInvalidValue;
+  p.gx = static_cast<const bf16*>(a.xp);
   p.grow = a.gather.rows;
   p.gk = a.gather.k;
   p.grows = static_cast<int>(a.rows);
@@ -1131,6 +1206,7 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.w1 = a.dWu;
   p.w2 = a.dWd;
   p.accumulate = a.accumulate;
+  p.gx = static_cast<const bf16*>(a.xp);
   p.grow = a.gather.rows;
   p.gk = a.gather.k;
   p.grows = static_cast<int>(a.rows);

@@ -115,6 +115,23 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same for shared memory written by cp.async copies whose completion this
+// thread has observed through an mbarrier (all state spaces).
+__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
+
+// 16-byte global -> shared copy through L2 (cp.async.cg), asynchronous.
+__device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+
+// Arrival on `bar` once every cp.async this thread issued so far has landed
+// (.noinc: the barrier's expected count includes this arrival).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ----------------------------------------------------------------- tcgen05
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -197,8 +214,6 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrive on an mbarrier given by its shared::cluster address (possibly in
-// the peer CTA).
 // 16 zero bytes at a shared::cluster address (this CTA's or a peer's).
 __device__ __forceinline__ void st_cluster_zero16(uint32_t cluster_addr) {
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(cluster_addr), "r"(0u)
@@ -211,6 +226,8 @@ __device__ __forceinline__ void fence_proxy_async_cluster() {
   asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
 
+// Arrive on an mbarrier given by its shared::cluster address (possibly in
+// the peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
@@ -218,20 +235,6 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 
 // TMA load into this CTA's shared memory whose completion is counted on the
 // mbarrier at `bar_cluster_addr`, which may live in the peer CTA of the pair.
-// TMA gather of four rows: rows r0..r3 of a 2D tensor, columns c0 .. c0 + box
-// width, into four consecutive rows of `dst` (the tensor map's box is one row
-// high). A pair's load counts on the even CTA's barrier at `bar_cluster_addr`.
-__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map,
-                                                 uint32_t bar_cluster_addr, int c0, int r0, int r1,
-                                                 int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4"
-      ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map,
                                                  uint32_t bar_cluster_addr, int c0, int c1) {
   asm volatile(

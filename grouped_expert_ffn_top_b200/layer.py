@@ -4,16 +4,18 @@ Forward:  moe_router_logits -> moe_route -> moe_permute -> moe_grouped_ffn_fwd
           -> moe_unpermute_combine
 Backward: moe_unpermute_combine_bwd -> moe_route_bwd -> moe_grouped_ffn_dgrad
           -> moe_grouped_ffn_wgrad -> moe_permute_bwd (with the router's input
-          gradient) -> moe_router_bwd
+          gradient) -> moe_router_bwd_gather (dispatch rows read from x)
 With checkpoint=True the forward does not store h1 and h2 and the backward
 first rebuilds them with moe_grouped_ffn_recompute (activation checkpointing:
 2 T k f activation elements less to keep between forward and backward, for
 one more gate/up GEMM).
-With fused_dispatch=True there is no permuted copy xp: the gate/up GEMM, the
-weight gradient's dWg / dWu operand and the router backward read dispatch
-row r in place as x[pair_of_row[r] / k] (moe_grouped_ffn_fwd_gather,
-moe_grouped_ffn_wgrad_gather, moe_router_bwd_gather), with results bitwise
-those of the permuted path; x must then stay unchanged until the backward.
+With fused_dispatch=True there is no permuted copy xp: the gate/up GEMM and
+the weight gradient's dWg / dWu operand read dispatch row r in place as
+x[pair_of_row[r] / k] (moe_grouped_ffn_fwd_gather,
+moe_grouped_ffn_wgrad_gather), with results bitwise those of the permuted
+path. It saves the T k d copy but is slower on this shape: the GEMMs re-read
+each row many times, and row-sized gathers move those re-reads at a fraction
+of the tiled loads' rate. Either way x must stay unchanged until the backward.
 With a balance-loss coefficient (aux_coef > 0) the forward also calls
 moe_aux_loss after routing, and the backward ends with moe_aux_loss_bwd ->
 moe_router_bwd_dense (the loss's dense logit gradient into dX, dWr, db).
@@ -209,14 +211,11 @@ class MoELayer:
         N.moe_permute_bwd(v["dxp"], r["row_of_pair"], v["dlogits"], self.Wr, r["topk_idx"], T, self.k,
                           dX, stream)
         mark("permute_bwd")
-        if self.fused:
-            N.moe_router_bwd_gather(self.x, v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"],
-                                    g["db"], self.ws["router_bwd"], stream, accumulate=accumulate)
-            mark("router_bwd_gather")
-        else:
-            N.moe_router_bwd(v["xp"], v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"], g["db"],
-                             self.ws["router_bwd"], stream, accumulate=accumulate)
-            mark("router_bwd")
+        # the router's weight gradient reads the dispatch rows from x (T d
+        # elements, k times fewer than xp) in both layouts: bitwise the same sums
+        N.moe_router_bwd_gather(self.x, v["dlogits"], r["pair_of_row"], r["offsets"], self.k, g["dWr"],
+                                g["db"], self.ws["router_bwd"], stream, accumulate=accumulate)
+        mark("router_bwd_gather")
         if self.aux_coef:
             N.moe_aux_loss_bwd(v["logits"], r["counts"], self.k, self.aux_coef, aux_dloss, v["dz_aux"],
                                stream)

@@ -230,7 +230,11 @@ MOE_API int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, 
  * moe_grouped_ffn_fwd; xp is neither written nor read.
  *   x [T, d] dtype; pair_of_row [T*k] int32 (moe_route's output); rows = T*k;
  *   every other argument and error as moe_grouped_ffn_fwd (k in 1..32).
- * The bf16 path loads the rows with TMA tile::gather4 (four rows a load). */
+ * The bf16 path gathers the rows with 16-byte cp.async copies into the
+ * GEMM's swizzled operand stages (the weights still arrive by TMA). It saves
+ * the copy xp but runs slower than moe_permute + moe_grouped_ffn_fwd on
+ * large d and f: the GEMM reads each row once per 128 output columns, and
+ * row-sized gathers deliver those reads at a fraction of the tiled TMA rate. */
 MOE_API int moe_grouped_ffn_fwd_gather(const void* x, const int32_t* pair_of_row, int64_t T, int k,
                                        const void* Wg, const void* Wu, const void* Wd, int dtype,
                                        const int64_t* expert_offsets, int E, int d, int f,

@@ -1,5 +1,5 @@
 """Fused dispatch: the expert GEMMs and the router backward read the dispatch
-rows in place from x through pair_of_row (TMA tile::gather4 on the bf16 path)
+rows in place from x through pair_of_row (cp.async row gathers on the bf16 path)
 instead of from the permuted copy xp.
 
 Dispatch row r is x[pair_of_row[r] / k], the row the permute copies to xp[r],
