@@ -626,7 +626,7 @@ __device__ __forceinline__ bool wait_stage(uint64_t* full, uint64_t* gfull, int 
                                            uint32_t phase, volatile int* abort) {
   if (GATHER) {
     if (!wait_bounded(&gfull[stage], phase, abort, kWaitLimit)) return false;
-    fence_proxy_async_all();
+    fence_proxy_async_smem();
   }
   return wait_bounded(&full[stage], phase, abort, kWaitLimit);
 }
@@ -939,7 +939,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
           ok = false;
           break;
         }
-        fence_proxy_async_all();
+        fence_proxy_async_smem();
         if (lane == 0) mbar_arrive_cluster(full_leader + 8u * static_cast<uint32_t>(stage));
         __syncwarp();
         if (++stage == STAGES) {

@@ -158,8 +158,8 @@ static cudaError_t launch_router_logits_t(const T* x, const T* Wr, const float* 
   } else if (E <= 32) {
     router_logits_kernel<T, 32, 128><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else {
-    router_logits_kernel<T, 64, 128><<<dim3(gx, (E + 63) / 64), 128, 0, s>>>(x, Wr, b, Ttok, d,
-                                                                             E, z);
+    router_logits_kernel<T, 64, 64><<<dim3(gx, (E + 63) / 64), 64, 0, s>>>(x, Wr, b, Ttok, d,
+                                                                           E, z);
   }
   return cudaGetLastError();
 }

@@ -109,15 +109,13 @@ __device__ __forceinline__ void bulk_wait_group() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Makes this thread's generic-proxy shared-memory writes visible to the async
-// proxy (TMA, tcgen05.mma operand reads).
+// Makes this thread's generic-proxy shared-memory writes, and cp.async
+// copies whose completion it has observed through an mbarrier, visible to the
+// async proxy (TMA, tcgen05.mma operand reads). The CTA-scoped form: the
+// unscoped fence.proxy.async also orders global memory and costs far more.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-
-// The same for shared memory written by cp.async copies whose completion this
-// thread has observed through an mbarrier (all state spaces).
-__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
 // 16-byte global -> shared copy through L2 (cp.async.cg), asynchronous.
 __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src) {
