@@ -177,12 +177,21 @@ def oracle_inputs(w, seed: int = 0):
 
 
 def calibrate_sample(step, budget_s: float, T: int) -> int:
-    """Largest token count whose oracle step takes about budget_s seconds."""
-    n = 4
-    t0 = time.perf_counter()
-    step(n)
-    dt = max(time.perf_counter() - t0, 1e-3)
-    return int(max(1, min(T, n * budget_s / dt)))
+    """Token count whose oracle step takes about budget_s seconds: a linear
+    fit (fixed cost + cost per token) through two probe sizes."""
+    def timed(n):
+        t0 = time.perf_counter()
+        step(n)
+        return max(time.perf_counter() - t0, 1e-4)
+
+    step(2)  # first call: thread start-up and first touches of the weights
+    n0 = 8
+    t0 = timed(n0)
+    n1 = int(max(2 * n0, min(T, n0 * 0.25 * budget_s / t0)))
+    t1 = timed(n1)
+    per_token = max((t1 - t0) / (n1 - n0), 1e-9)
+    fixed = max(t0 - per_token * n0, 0.0)
+    return int(max(1, min(T, (budget_s - fixed) / per_token)))
 
 
 def cpu_baseline(w, budget_s: float = 15.0):
@@ -512,7 +521,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="fine_fwdbwd_32k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--checkpoint", action="store_true",
                     help="activation checkpointing: h1, h2 rebuilt in the backward")
     ap.add_argument("--dispatch", choices=["permute", "fused"], default="permute",
