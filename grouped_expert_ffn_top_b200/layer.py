@@ -21,7 +21,10 @@ moe_aux_loss after routing, and the backward ends with moe_aux_loss_bwd ->
 moe_router_bwd_dense (the loss's dense logit gradient into dX, dWr, db).
 
 The object owns device buffers sized for `max_tokens`, so a step allocates
-nothing; microbatches of any size up to that (0 included) reuse them. Weight
+nothing; microbatches of any size up to that (0 included) reuse them. No call
+synchronises with the host, so forward + backward on fixed input buffers can be
+captured once into a CUDA graph and replayed for every new batch of that size
+(the routing, expert offsets and GEMM tile lists all live on the device). Weight
 gradients accumulate in fp32 across microbatches until zero_grad(); a
 backward with accumulate=False writes them instead (the first microbatch of a
 step: the old values are neither read nor needed).
