@@ -364,6 +364,7 @@ class Ranks:
 # ------------------------------------------------------------ native arm
 
 def run_native(args, w):
+    import numpy as np
     import torch
 
     from grouped_expert_ffn_top_b200 import native as N
@@ -443,6 +444,18 @@ def run_native(args, w):
     if errs:
         raise RuntimeError(f"device error word {errs} in the timed region")
 
+    # routing load of the batch and the device memory the step held (read
+    # after the timed regions)
+    counts = layer.r["counts"].cpu().numpy().astype(np.int64)
+    nonzero = counts[counts > 0]
+    routing = {"experts": int(counts.size), "empty_experts": int((counts == 0).sum()),
+               "rows_max": int(counts.max()), "rows_min_nonzero": int(nonzero.min()) if nonzero.size else 0,
+               "max_over_mean": round(float(counts.max() / max(counts.mean(), 1e-9)), 3)}
+    free_b, total_b = torch.cuda.mem_get_info(dev)
+    memory = {"peak_allocated_gb": round(torch.cuda.max_memory_allocated(dev) / 1e9, 2),
+              "device_used_gb": round((total_b - free_b) / 1e9, 2),
+              "device_total_gb": round(total_b / 1e9, 1)}
+
     hbm, bf16_burst, bf16_sust, peak_src = _peaks()
     flops, bytes_ = algorithmic_work(w, T)
     kernels = {}
@@ -500,6 +513,8 @@ def run_native(args, w):
                        "copies run on two copy streams, double-buffered so step i+1's inputs "
                        "arrive while step i computes"},
         "gpu_launches": int(launches),
+        "routing": routing,
+        "memory": memory,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
