@@ -1,0 +1,51 @@
+"""bench.py's host-side logic on the CPU: the sizing of the oracle sample, the
+algorithmic work the roofline divides by, and the workload description."""
+import bench
+from grouped_expert_ffn_top_b200 import workloads
+
+
+def _fake_clock(monkeypatch, fixed, per_token):
+    clock = [0.0]
+    monkeypatch.setattr(bench.time, "perf_counter", lambda: clock[0])
+
+    def step(n):
+        clock[0] += fixed + per_token * n
+
+    return step
+
+
+def test_oracle_sample_fits_fixed_and_per_token_cost(monkeypatch):
+    # a step of n tokens costs 0.5 s + 0.1 s per token: 145 tokens fill 15 s
+    step = _fake_clock(monkeypatch, 0.5, 0.1)
+    assert abs(bench.calibrate_sample(step, 15.0, 32768) - 145) <= 1
+
+
+def test_oracle_sample_is_clamped_to_the_batch(monkeypatch):
+    step = _fake_clock(monkeypatch, 0.0, 1e-6)
+    assert bench.calibrate_sample(step, 15.0, 1000) == 1000
+    step = _fake_clock(monkeypatch, 100.0, 1.0)  # even one token is over budget
+    assert bench.calibrate_sample(step, 15.0, 1000) == 1
+
+
+def test_algorithmic_work_of_the_bench_workload():
+    w = workloads.WORKLOADS["fine_fwdbwd_32k"]
+    T = w.T[0]
+    P = T * w.k
+    flops, bytes_ = bench.algorithmic_work(w, T)
+    # each grouped GEMM call: three d x f products per dispatched row
+    for n in ("grouped_ffn_fwd", "grouped_ffn_dgrad", "grouped_ffn_wgrad"):
+        assert flops[n] == 6.0 * w.d * w.f * P
+    # the fused-dispatch forms do the same arithmetic
+    for n in ("grouped_ffn_fwd", "grouped_ffn_wgrad", "router_bwd"):
+        assert flops[n + "_gather"] == flops[n]
+    assert flops["router_logits"] == 2.0 * T * w.d * w.E
+    # permute: x read once, k copies written, the row map read
+    assert bytes_["permute"] == (T * w.d + P * w.d) * 2 + 4 * P
+
+
+def test_workload_config_names_the_shape():
+    w = workloads.WORKLOADS["fine_fwdbwd_32k"]
+    c = bench.workload_config(w)
+    assert c["workload"] == "fine_fwdbwd_32k"
+    assert (c["tokens_per_gpu"], c["d_model"], c["experts"], c["top_k"], c["ffn"]) == (32768, 2048, 64, 8, 1408)
+    assert "l2" in c
