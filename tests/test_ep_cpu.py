@@ -1,5 +1,6 @@
-"""Expert parallelism on the CPU: two gloo ranks, experts sharded 4 + 4, with
-uneven and empty microbatches and a local expert that receives no rows. The
+"""Expert parallelism on the CPU: two and four gloo ranks (experts sharded
+4 + 4, or 2 + 2 + 2 + 2), with uneven and empty microbatches and local experts
+that receive no rows. The
 layer's exchange logic (count all-to-all, ragged row all-to-alls, regroup by
 local expert and back) runs as in production; the local steps run in the
 oracle (test-only `OracleOps`), so every rank's Y and dX must equal the
@@ -168,12 +169,16 @@ def _free_port():
     return p
 
 
-@pytest.mark.parametrize("Ts", [(37, 0), (20, 13)])
-def test_two_rank_expert_parallel_layer_matches_oracle(Ts):
+@pytest.mark.parametrize("Ts", [(37, 0), (20, 13), (25, 0, 9, 1)],
+                         ids=["2 ranks, one empty", "2 ranks", "4 ranks, uneven, one empty"])
+def test_expert_parallel_layer_matches_oracle(Ts):
+    """World size len(Ts): 2 ranks with experts sharded 4 + 4, and 4 ranks
+    (expert groups of 2, the group count of the 32k workload's layout)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, Ts, q)) for r in range(2)]
+    world = len(Ts)
+    procs = [ctx.Process(target=_worker, args=(r, world, port, Ts, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = dict(q.get(timeout=180) for _ in procs)
