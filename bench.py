@@ -228,7 +228,7 @@ def run_reference(args, w):
         "warmup": args.warmup, "ms_per_step": 1000.0 * dt / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": workload_config(w),
+        "config": dict(workload_config(w), parallelism=f"dp{args.gpus}"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": f"each step: oracle fwd+bwd of the first {n} tokens"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -496,10 +496,12 @@ def run_native(args, w):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian activations and weights, Zipf-skewed router bias)",
         "impl": "native",
-        "config": dict(workload_config(w), parallelism=f"dp{world}",
-                       **({"checkpoint": "h1, h2 rebuilt in the backward"} if args.checkpoint else {}),
-                       dispatch=("fused: expert rows gathered from x inside the GEMM operand loads, "
-                                 "no permuted copy" if fused else "permute: rows copied to xp first")),
+        "config": dict(workload_config(w), parallelism=f"dp{world}"),
+        # how this arm runs the layer (the workload is the same either way)
+        "options": {"dispatch": ("fused: expert rows gathered from x inside the GEMM operand loads, "
+                                 "no permuted copy" if fused else "permute: rows copied to xp first"),
+                    "activations": ("checkpointed: h1, h2 rebuilt in the backward" if args.checkpoint
+                                    else "stored")},
         "grouped_gemm": {"tflops": round(gemm_tf, 1), "frac_bf16_sustained": round(gemm_tf / bf16_sust, 3),
                          "frac_bf16_burst": round(gemm_tf / bf16_burst, 3)},
         "permute_combine": {"gbs": round(mem_gbs, 1), "frac_hbm": round(mem_gbs / hbm, 3),
