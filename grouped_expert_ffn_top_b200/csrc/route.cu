@@ -254,22 +254,26 @@ __global__ void __launch_bounds__(NT) topk_softmax_kernel(
         my_idx = best.idx;
       }
     }
-    // softmax over the k selected logits (fp32)
+    // softmax over the k selected logits (fp32), exp(z_j - m) / sum with m
+    // the largest selected logit; a selected -inf next to a finite m gets
+    // exactly 0. It is undefined only when m is not finite (+inf - +inf, or
+    // every selected logit -inf) or a selected logit is NaN (NaN ranks last,
+    // so the k-th is then NaN): those tokens get 1/k and raise the flag.
     const bool active = lane < k;
-    const bool finite = !active || isfinite(my_val);
-    const bool all_finite = __all_sync(0xffffffffu, finite);
     const float m = __shfl_sync(0xffffffffu, my_val, 0);
-    float ex = (active && all_finite) ? expf(my_val - m) : 0.0f;
+    const float last = __shfl_sync(0xffffffffu, my_val, k - 1);
+    const bool defined = isfinite(m) && !isnan(last);
+    float ex = (active && defined) ? expf(my_val - m) : 0.0f;
     float sum = ex;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     if (active) {
-      const float w = all_finite ? ex / sum : 1.0f / static_cast<float>(k);
+      const float w = defined ? ex / sum : 1.0f / static_cast<float>(k);
       topk_idx[t * k + lane] = my_idx;
       topk_w[t * k + lane] = w;
       atomicAdd(&s_hist[my_idx], 1);
     }
-    if (!all_finite && lane == 0) raise_error(err, kErrNonfiniteLogit);
+    if (!defined && lane == 0) raise_error(err, kErrNonfiniteLogit);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)

@@ -79,7 +79,7 @@ extern "C" {
 #define MOE_ERR_CUDA (-4)        /* a CUDA call or launch failed              */
 
 /* Bits of the device error word returned by moe_get_error. */
-#define MOE_DEVERR_NONFINITE_LOGIT 1u /* a selected router logit was NaN or +-inf */
+#define MOE_DEVERR_NONFINITE_LOGIT 1u /* a token's gate softmax was undefined   */
 #define MOE_DEVERR_TIMEOUT 2u         /* a bounded wait inside a kernel gave up   */
 
 /* Limits of this build. */
@@ -130,9 +130,11 @@ MOE_API size_t moe_route_workspace_bytes(int64_t T, int E);
 /* Top-k softmax routing and the dispatch layout, all on the device.
  * Selection: per token the k largest logits, ties to the lower expert index,
  * NaN below every number, slots in descending order. Gate weights: softmax
- * over the k selected logits (they sum to 1). If a selected logit is not
- * finite the token's weights are 1/k each and MOE_DEVERR_NONFINITE_LOGIT is
- * raised in the ws error word.
+ * over the k selected logits (they sum to 1), exp(z_j - m) / sum_i
+ * exp(z_i - m) with m the largest selected logit; a selected -inf next to a
+ * finite m gets exactly 0. Where that softmax is undefined -- m is +inf, every
+ * selected logit is -inf, or a selected logit is NaN -- the token's weights
+ * are 1/k each and MOE_DEVERR_NONFINITE_LOGIT is raised in the ws error word.
  * Layout (EP token dispatch, leap-finetune PR #26 Summary; expert
  * communication groups, ART issue #917 Desired behavior): pair (t,j) gets
  * row row_of_pair[t*k+j]; rows are sorted by (expert, token), both

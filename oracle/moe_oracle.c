@@ -42,7 +42,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define ORC_FLAG_NONFINITE 1 /* a selected logit was NaN or +-inf */
+#define ORC_FLAG_NONFINITE 1 /* a softmax over the selected logits was undefined */
 
 /* ---------------------------------------------------------------- router */
 
@@ -87,8 +87,13 @@ static int ranks_before(double za, int ia, double zb, int ib) {
 /* Top-k selection and gate weights per token.
  * topk_idx[t,j] is the j-th ranked expert; topk_w[t,j] = softmax over the k
  * selected logits (equivalently, the softmax over all E renormalised to the
- * selected k). If a selected logit is not finite the weights are 1/k each and
- * the returned flag word has ORC_FLAG_NONFINITE set.
+ * selected k), computed as exp(z_j - m) / sum_i exp(z_i - m) with m the
+ * largest selected logit. A selected -inf next to a finite m is well defined
+ * and gets exactly 0. The softmax is undefined only when m is not finite
+ * (+inf gives inf - inf; m = -inf means every selected logit is -inf, 0/0)
+ * or a selected logit is NaN (NaN ranks last, so then the k-th one is NaN):
+ * only then are the weights 1/k each and the returned flag word has
+ * ORC_FLAG_NONFINITE set.
  * Reads z in double (an fp32 logit converts exactly). */
 int orc_route(const double* z, int64_t T, int E, int k, int32_t* topk_idx, double* topk_w) {
   int flags = 0;
@@ -107,17 +112,13 @@ int orc_route(const double* z, int64_t T, int E, int k, int32_t* topk_idx, doubl
         }
         order[p] = e;
       }
-      int finite = 1;
-      for (int j = 0; j < k; ++j) {
-        topk_idx[t * k + j] = order[j];
-        if (!isfinite(zt[order[j]])) finite = 0;
-      }
-      if (!finite) {
+      for (int j = 0; j < k; ++j) topk_idx[t * k + j] = order[j];
+      const double m = zt[order[0]];
+      if (!isfinite(m) || isnan(zt[order[k - 1]])) {
         flags |= ORC_FLAG_NONFINITE;
         for (int j = 0; j < k; ++j) topk_w[t * k + j] = 1.0 / k;
         continue;
       }
-      double m = zt[order[0]];
       double s = 0.0;
       for (int j = 0; j < k; ++j) s += exp(zt[order[j]] - m);
       for (int j = 0; j < k; ++j) topk_w[t * k + j] = exp(zt[order[j]] - m) / s;

@@ -42,9 +42,15 @@ def test_route_bitexact_on_tied_logits(T, E, k, G):
 
 
 def test_route_nonfinite_logits_raise_the_device_flag():
+    inf, nan = float("inf"), float("nan")
     z = workloads.make_logits(300, 16, seed=5, specials=True)
-    z[7, :] = -float("inf")
-    z[9, 3] = float("nan")
+    z[7, :] = -inf                       # all selected -inf: undefined, 1/k
+    z[9, 3] = nan                        # NaN outside the selection: ignored
+    z[11, :] = -inf
+    z[11, 2], z[11, 5] = 1.0, 2.0        # two finite then -inf: defined, zeros
+    z[13, 4] = inf                       # +inf selected: undefined
+    z[15, :] = nan
+    z[15, 0] = 0.5                       # NaN selected: undefined
     ws = N._ws(N.moe_route_workspace_bytes(300, 16), DEV)
     out = N.moe_route(z.to(DEV), 4, 1, ws=ws)
     assert N.moe_get_error(ws) & N.MOE_DEVERR_NONFINITE_LOGIT
@@ -52,7 +58,26 @@ def test_route_nonfinite_logits_raise_the_device_flag():
     idx, w, flags = oracle.route(z.double().numpy(), 4)
     assert flags & oracle.FLAG_NONFINITE
     assert np.array_equal(to_np(out["topk_idx"]), idx)
-    assert np.array_equal(to_np(out["topk_w"])[7], np.full(4, 0.25, np.float32))
+    gw = to_np(out["topk_w"])
+    assert np.abs(gw - w).max() <= 1e-6
+    for t in (7, 13, 15):
+        assert np.array_equal(gw[t], np.full(4, 0.25, np.float32)), t
+    assert gw[11, 2] == 0.0 and gw[11, 3] == 0.0 and abs(gw[11, 0] - 0.7310586) < 1e-6
+
+
+def test_route_with_selected_minus_inf_is_a_defined_softmax():
+    """-inf logits inside the selection next to finite ones: exact softmax
+    (zero weight on the -inf slots), no device flag."""
+    z = workloads.make_logits(500, 8, seed=6)
+    z[::3, 2:] = -float("inf")           # only experts 0 and 1 finite, k = 4
+    ws = N._ws(N.moe_route_workspace_bytes(500, 8), DEV)
+    out = N.moe_route(z.to(DEV), 4, 2, ws=ws)
+    assert N.moe_get_error(ws) == 0
+    idx, w, flags = oracle.route(z.double().numpy(), 4)
+    assert flags == 0
+    lay = oracle.dispatch_layout(idx, 8, 2)
+    check_routing_bitexact(out, None, dict(idx=idx, w=w, **lay), check_logits=False)
+    assert not to_np(out["topk_w"])[::3, 2:].any()
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])

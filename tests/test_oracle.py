@@ -104,7 +104,31 @@ def test_route_nan_ranks_last_and_nonfinite_flags():
     idx, w, flags = oracle.route(z, 3)
     assert idx.tolist() == [[3, 1, 2], [0, 3, 1], [2, 3, 0]]
     assert flags & oracle.FLAG_NONFINITE
-    assert np.all(w == 1.0 / 3)
+    # selected (2, 1, -inf): the softmax is defined; by hand e^0 / (1 + e^-1)
+    # = 0.7310586, e^-1 / (1 + e^-1) = 0.2689414, and exactly 0 for -inf
+    np.testing.assert_allclose(w[0], [0.7310585786300049, 0.2689414213699951, 0.0], rtol=1e-15)
+    assert w[0, 2] == 0.0
+    # selected (0, -1, NaN): undefined, 1/k each
+    assert np.all(w[1] == 1.0 / 3)
+    # selected (3, 1, -inf): e^0 / (1 + e^-2) = 0.8807971, e^-2 / (1 + e^-2) = 0.1192029
+    np.testing.assert_allclose(w[2], [0.8807970779778823, 0.11920292202211755, 0.0], rtol=1e-15)
+
+
+def test_route_undefined_softmax_falls_back_to_uniform_weights():
+    inf = np.inf
+    # all selected -inf (0/0), +inf selected (inf - inf), NaN selected
+    for row, k in (([-inf, -inf, -inf, -inf], 2), ([inf, 1.0, 0.0, 2.0], 2),
+                   ([inf, inf, 0.0, 2.0], 3), ([1.0, np.nan, np.nan, np.nan], 2)):
+        idx, w, flags = oracle.route(np.array([row]), k)
+        assert flags & oracle.FLAG_NONFINITE, row
+        assert np.all(w == 1.0 / k), row
+    # one finite logit with -inf after it: the whole weight on the finite one
+    idx, w, flags = oracle.route(np.array([[-inf, 0.25, -inf, -inf]]), 3)
+    assert flags == 0
+    assert idx.tolist() == [[1, 0, 2]] and w.tolist() == [[1.0, 0.0, 0.0]]
+    # a NaN outside the selection does not matter
+    idx, w, flags = oracle.route(np.array([[np.nan, 1.0, 1.0, 0.0]]), 2)
+    assert flags == 0 and idx.tolist() == [[1, 2]] and w.tolist() == [[0.5, 0.5]]
 
 
 def test_route_weights_properties(rng):
