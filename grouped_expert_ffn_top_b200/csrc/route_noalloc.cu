@@ -11,12 +11,16 @@
 // library holds its own copy (MOE_ROUTE_NOALLOC_MAX_SLOTS * 8 bytes, 2 MiB)
 // until the process exits. Host code cannot use the variable's name as a
 // device address, so the first call on each device looks the address up
-// with cudaGetSymbolAddress (with that device current) and caches it; make
-// that first call before any stream capture. All calls on a device share the
+// with cudaGetSymbolAddress (with that device current) and caches it with the
+// id of the device's current context; make that first call before any stream
+// capture. A later call in another context (after cudaDeviceReset the module
+// is loaded again, at a new address) looks it up again. All calls on a device share the
 // one array, so calls that overlap on the GPU (different streams, or
 // concurrent host threads) race and must be serialised by the caller. Every
 // entry the kernels read is written earlier in the same call, so nothing has
 // to be cleared between calls.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -31,8 +35,38 @@ static __device__ __align__(256) int32_t g_route_scratch[2 * MOE_ROUTE_NOALLOC_M
 
 std::mutex g_mu;
 int32_t* g_scratch_of_device[kMaxDevices] = {};
+unsigned long long g_ctx_of_device[kMaxDevices] = {};
 
-// Device address of this device's copy of the array (looked up once).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of this device's copy of the array: looked up on the first
+// call on the device and again whenever the device's context has changed.
 int scratch_for_current_device(int32_t** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -41,12 +75,23 @@ int scratch_for_current_device(int32_t** out) {
   if (dev < 0 || dev >= kMaxDevices)
     return moe::report_error(MOE_ERR_UNSUPPORTED, "moe_route_noalloc: device index out of range");
   std::lock_guard<std::mutex> lock(g_mu);
+  // makes the device's primary context current if no call has yet
+  void* p = nullptr;
   if (!g_scratch_of_device[dev]) {
-    void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess || !p)
       return moe::report_error(MOE_ERR_CUDA, "moe_route_noalloc: cudaGetSymbolAddress failed");
     g_scratch_of_device[dev] = static_cast<int32_t*>(p);
+    g_ctx_of_device[dev] = current_context_id();
+  } else {
+    const unsigned long long ctx = current_context_id();
+    if (ctx == 0 || ctx != g_ctx_of_device[dev]) {
+      e = cudaGetSymbolAddress(&p, g_route_scratch);
+      if (e != cudaSuccess || !p)
+        return moe::report_error(MOE_ERR_CUDA, "moe_route_noalloc: cudaGetSymbolAddress failed");
+      g_scratch_of_device[dev] = static_cast<int32_t*>(p);
+      g_ctx_of_device[dev] = ctx;
+    }
   }
   *out = g_scratch_of_device[dev];
   return MOE_OK;

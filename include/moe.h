@@ -182,7 +182,10 @@ MOE_API int moe_route(const float* logits, int64_t T, int E, int k, int ep_group
  *   - err_flags: device pointer to a caller-zeroed unsigned int that the
  *     kernels OR MOE_DEVERR_* bits into, or NULL to not report them.
  * The first call on each device looks up the array's device address (with
- * that device current); make it before any stream capture. All calls on a
+ * that device current); make it before any stream capture. The address is
+ * kept per device ordinal and looked up again when the device's primary
+ * context changes (after cudaDeviceReset the array lives at a new address
+ * in the new context). All calls on a
  * device share the array: calls that overlap on the GPU (other streams,
  * other host threads) race, so the caller must serialise them. Nothing has
  * to be cleared between calls. */

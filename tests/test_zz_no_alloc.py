@@ -5,10 +5,14 @@ forbid allocations after planning, paths where cudaMalloc's implicit device
 synchronisation is not allowed) cannot hand moe_route a workspace; this entry
 point uses a fixed array inside the library instead. The test calls it
 through the C ABI twice in a row, on different logits, and checks every
-output against moe_route on the same input. It also runs alone in a fresh
-process: the first call on the device performs the one-time address lookup.
+output against moe_route on the same input. Run after the other GPU tests, the
+array's address was looked up by an earlier call in this process; the last
+test repeats the same check in a fresh Python process, where the first call
+on the device makes that lookup.
 """
-import ctypes
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -63,3 +67,14 @@ def test_noalloc_route_reports_flags_and_limits():
     rc, _ = _noalloc(big, 2, 1, None)
     assert rc == N.MOE_ERR_UNSUPPORTED
     assert b"MOE_ROUTE_NOALLOC_MAX_SLOTS" in N.lib().moe_last_error()
+
+
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="no CUDA device")
+def test_noalloc_route_in_a_fresh_process():
+    here = os.path.dirname(os.path.abspath(__file__))
+    code = ("import sys; sys.path[:0] = [%r, %r]; "
+            "import test_zz_no_alloc as t; t.test_noalloc_route_equals_moe_route_on_two_calls(); "
+            "print('fresh process ok')" % (here, os.path.dirname(here)))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "fresh process ok" in r.stdout
