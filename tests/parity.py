@@ -44,6 +44,31 @@ def assert_close(name: str, gpu, ref, tol: float):
     return e
 
 
+def rel_err_per(gpu, ref) -> float:
+    """Worst over the leading index (a token, a dispatch row, an expert) of
+    max|gpu - ref| / max|ref| taken within that slice, so a wrong result in a
+    small slice cannot hide under the largest slice's magnitude. A slice whose
+    reference is all zero is measured against the whole tensor's scale."""
+    g = to_np(gpu).astype(np.float64) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, np.float64)
+    r = np.asarray(ref, np.float64)
+    if r.size == 0:
+        return 0.0
+    n = r.shape[0]
+    g = g.reshape(n, -1)
+    r = r.reshape(n, -1)
+    glob = np.abs(r).max()
+    scale = np.abs(r).max(axis=1)
+    scale = np.where(scale > 0.0, scale, glob if glob > 0.0 else 1.0)
+    return float((np.abs(g - r).max(axis=1) / scale).max())
+
+
+def assert_close_per(name: str, gpu, ref, tol: float):
+    """assert_close with the scale taken per leading index (rel_err_per)."""
+    e = rel_err_per(gpu, ref)
+    assert e <= tol, f"{name}: max relative error per slice {e:.3e} > {tol:.1e}"
+    return e
+
+
 def oracle_routing(x: torch.Tensor, Wr: torch.Tensor, b: torch.Tensor, k: int, G: int):
     """Oracle logits (fp32 fixed order), top-k and layout for all tokens."""
     z = oracle.router_logits_f32(to_np(x).astype(np.float32), to_np(Wr).astype(np.float32),
@@ -65,11 +90,14 @@ def check_routing_bitexact(layer_route: Dict[str, torch.Tensor], logits_gpu: tor
 
 def sampled_forward_backward(x, dY, params, ref_route: dict, tokens: np.ndarray, k: int,
                              backward: bool = True):
-    """Oracle Y (and dX) for the given tokens, one expert at a time.
+    """Oracle Y (and dX, dg, dlogits) for the given tokens, one expert at a time.
 
-    Y_t = sum_j g_{t,j} FFN_{S_{t,j}}(x_t); the expert part of dX for each pair
-    comes from the per-token oracle with that pair alone, the router part from
-    oracle.route_bwd / oracle.router_bwd over the token's k slots."""
+    Each pair's expert output y_{t,j} = FFN_{S_{t,j}}(x_t) comes from the
+    per-token oracle (one expert's weights at a time); the sample's pairs are
+    then laid out as dispatch rows in (token, slot) order, and Y and dg come
+    from oracle.combine / oracle.combine_bwd over them. The expert part of dX
+    of each pair is the per-token oracle's backward of that pair alone, the
+    router part oracle.route_bwd / oracle.router_bwd over the token's k slots."""
     E = params["Wg"].shape[0]
     d = x.shape[1]
     xs = to_np(x[torch.as_tensor(tokens, dtype=torch.long, device=x.device)]).astype(np.float64)
@@ -78,9 +106,8 @@ def sampled_forward_backward(x, dY, params, ref_route: dict, tokens: np.ndarray,
     idx = ref_route["idx"][tokens]
     w = ref_route["w"][tokens]
     n = len(tokens)
-    Y = np.zeros((n, d))
+    ys_all = np.zeros((n, k, d))
     dX = np.zeros((n, d))
-    dg = np.zeros((n, k))
     for e in np.unique(idx):
         sel_t, sel_j = np.nonzero(idx == e)
         Wg = to_np(params["Wg"][e:e + 1]).astype(np.float64)
@@ -89,13 +116,16 @@ def sampled_forward_backward(x, dY, params, ref_route: dict, tokens: np.ndarray,
         one = np.zeros((len(sel_t), 1), np.int32)
         g = w[sel_t, sel_j][:, None]
         _, ys = oracle.tokens_fwd(xs[sel_t], one, np.ones_like(g), Wg, Wu, Wd)
-        Y[sel_t] += g * ys[:, 0, :]
+        ys_all[sel_t, sel_j] = ys[:, 0, :]
         if backward:
-            dg[sel_t, sel_j] = np.einsum("nd,nd->n", dYs[sel_t], ys[:, 0, :])
             _, dXe = oracle.tokens_bwd(xs[sel_t], dYs[sel_t], one, g, ys, np.zeros((1, d)), Wg, Wu, Wd)
             np.add.at(dX, sel_t, dXe)
-    out = {"Y": Y}
+    # the sample's pairs as dispatch rows in (token, slot) order
+    yp = ys_all.reshape(n * k, d)
+    rop = np.arange(n * k, dtype=np.int32)
+    out = {"Y": oracle.combine(yp, w, rop)}
     if backward:
+        _, dg = oracle.combine_bwd(dYs, yp, w, rop)
         dz = oracle.route_bwd(dg, w, idx, E)
         Wr = to_np(params["Wr"]).astype(np.float64)
         dX, _, _ = oracle.router_bwd(xs, Wr, dz, dX)

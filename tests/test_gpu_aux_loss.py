@@ -8,7 +8,7 @@ import oracle
 from grouped_expert_ffn_top_b200 import native as N
 from grouped_expert_ffn_top_b200 import workloads
 from grouped_expert_ffn_top_b200.layer import MoELayer
-from parity import TOL, assert_close, oracle_routing, rel_err, to_np
+from parity import TOL, assert_close, assert_close_per, oracle_routing, rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -138,3 +138,17 @@ def test_checkpointed_backward_is_bitwise_the_stored_one(dtype):
         assert torch.equal(ref.v[n], ck.v[n]), n
     for n in ref.grads:
         assert torch.equal(ref.grads[n], ck.grads[n]), n
+    # and the checkpointed layer itself against the oracle
+    tol = TOL[w.torch_dtype()]
+    P = {n: to_np(v).astype(np.float64) for n, v in p.items()}
+    x64 = to_np(bt["x"]).astype(np.float64)
+    fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k, 2)
+    bw = oracle.layer_backward(fw, x64, to_np(bt["dY"]).astype(np.float64), P["Wr"], P["Wg"], P["Wu"],
+                               P["Wd"], k)
+    assert_close_per("Y", Y1, fw["Y"], tol)
+    assert_close_per("dX", dX1, bw["dX"], tol)
+    for n in ("h1", "h2"):
+        assert_close_per(n, ck.v[n], fw[n], tol)
+    for n in ("dWg", "dWu", "dWd", "dWr"):
+        assert_close_per(n, ck.grads[n], bw[n], tol)
+    assert_close("db", ck.grads["db"], bw["db"], tol)

@@ -1,9 +1,11 @@
 """Expert parallelism on one GPU: with one rank the expert-parallel layer's
 exchanges are identities, so through the library's kernels it must give the
 plain layer's results bit for bit, with no process group and through a
-one-rank NCCL group (which runs the real all-to-all calls)."""
+one-rank NCCL group (which runs the real all-to-all calls); and its results
+must match the oracle's layer directly."""
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
@@ -12,6 +14,9 @@ from grouped_expert_ffn_top_b200 import native as N
 from grouped_expert_ffn_top_b200 import workloads
 from grouped_expert_ffn_top_b200.ep import EPMoELayer
 from grouped_expert_ffn_top_b200.layer import MoELayer
+
+import oracle
+from parity import TOL, assert_close, assert_close_per, to_np
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -56,6 +61,18 @@ def _compare(with_group: bool):
     assert torch.equal(dX0, dX1)
     for n in ref.grads:
         assert torch.equal(ref.grads[n], ep.grads[n]), n
+    # the expert-parallel layer against the oracle's layer
+    tol = TOL[torch.bfloat16]
+    P = {n: to_np(v).astype(np.float64) for n, v in p.items()}
+    x64 = to_np(bt["x"]).astype(np.float64)
+    fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k)
+    bw = oracle.layer_backward(fw, x64, to_np(bt["dY"]).astype(np.float64), P["Wr"], P["Wg"], P["Wu"],
+                               P["Wd"], k)
+    assert_close_per("Y", Y1, fw["Y"], tol)
+    assert_close_per("dX", dX1, bw["dX"], tol)
+    for n in ("dWg", "dWu", "dWd", "dWr"):
+        assert_close_per(n, ep.grads[n], bw[n], tol)
+    assert_close("db", ep.grads["db"], bw["db"], tol)
 
 
 def test_one_rank_expert_parallel_layer_is_the_plain_layer():
