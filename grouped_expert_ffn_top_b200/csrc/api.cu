@@ -245,6 +245,17 @@ int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dl
                      "moe_permute_bwd") == MOE_OK ? launched(MOE_OK, 1) : MOE_ERR_CUDA;
 }
 
+int moe_ep_regroup(const int32_t* recv_counts, int G, int El, int32_t* row_map,
+                   int64_t* local_offsets, cudaStream_t stream) {
+  if (G < 1 || El < 1 || !recv_counts || !row_map || !local_offsets)
+    return fail(MOE_ERR_INVALID_ARG, "moe_ep_regroup: G=%d El=%d or null pointer", G, El);
+  if (static_cast<int64_t>(G) * El > MOE_MAX_EXPERTS)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_ep_regroup: G*El=%lld > %d", static_cast<long long>(G) * El,
+                MOE_MAX_EXPERTS);
+  return cuda_status(moe::launch_ep_regroup(recv_counts, G, El, row_map, local_offsets, stream),
+                     "moe_ep_regroup") == MOE_OK ? launched(MOE_OK, 1) : MOE_ERR_CUDA;
+}
+
 size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E) {
   if (rows < 0 || d < 1 || E < 1) return 0;
   const size_t items = static_cast<size_t>(moe::router_bwd_max_items(rows, E));

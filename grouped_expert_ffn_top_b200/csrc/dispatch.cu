@@ -466,4 +466,58 @@ cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* po
   return cudaGetLastError();
 }
 
+// ------------------------------------------------- expert-parallel regroup
+// recv [G, El]: rows this rank received from source rank s for its local
+// expert e. They arrive sources ascending and, within a source, experts
+// ascending, so block (s, e) starts at received row
+//   A(s, e) = sum of the counts before (s, e) in row-major order,
+// and its row q goes to
+//   D(s, e) + q,  D(s, e) = sum_{e' < e} sum_s' recv[s', e'] + sum_{s' < s} recv[s', e],
+// which sorts the rows by (local expert, source rank, arrival). Local expert
+// e owns rows [local_offsets[e], local_offsets[e+1]). One block per (s, e);
+// each sums the G El <= MOE_MAX_EXPERTS counts it needs.
+__global__ void __launch_bounds__(256) ep_regroup_kernel(const int32_t* __restrict__ recv, int G, int El,
+                                                         int32_t* __restrict__ row_map,
+                                                         int64_t* __restrict__ local_offsets) {
+  const int blk = blockIdx.x;
+  const int s = blk / El, e = blk % El;
+  int64_t a = 0, dd = 0;
+  for (int i = threadIdx.x; i < G * El; i += blockDim.x) {
+    const int64_t c = recv[i];
+    const int si = i / El, ei = i % El;
+    if (i < blk) a += c;
+    if (ei < e || (ei == e && si < s)) dd += c;
+  }
+  __shared__ int64_t s_a[8], s_d[8];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, off);
+    dd += __shfl_xor_sync(0xffffffffu, dd, off);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    s_a[warp] = a;
+    s_d[warp] = dd;
+  }
+  __syncthreads();
+  a = 0;
+  dd = 0;
+  for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) {
+    a += s_a[w];
+    dd += s_d[w];
+  }
+  const int n = recv[blk];
+  for (int q = threadIdx.x; q < n; q += blockDim.x) row_map[a + q] = static_cast<int32_t>(dd + q);
+  if (threadIdx.x == 0) {
+    if (s == 0) local_offsets[e] = dd;
+    if (blk == G * El - 1) local_offsets[El] = a + n;
+  }
+}
+
+cudaError_t launch_ep_regroup(const int32_t* recv, int G, int El, int32_t* row_map,
+                              int64_t* local_offsets, cudaStream_t s) {
+  ep_regroup_kernel<<<G * El, 256, 0, s>>>(recv, G, El, row_map, local_offsets);
+  return cudaGetLastError();
+}
+
 }  // namespace moe

@@ -38,6 +38,9 @@ cudaError_t launch_combine_bwd(const void* dY, const void* yp, const float* w,
 cudaError_t launch_permute_bwd(const void* dxp, const int32_t* row_of_pair, const float* dz,
                                const void* Wr, const int32_t* idx, int dtype, int64_t T, int d,
                                int E, int k, void* dX, cudaStream_t s);
+// expert-parallel regroup of received rows (1 launch)
+cudaError_t launch_ep_regroup(const int32_t* recv, int G, int El, int32_t* row_map,
+                              int64_t* local_offsets, cudaStream_t s);
 int router_bwd_max_items(int64_t rows, int E);
 // gather: `xp` is x [T, d] and dispatch row r is read as x[pair_of_row[r] / k]
 cudaError_t launch_router_bwd(const void* xp, const float* dz, const int32_t* pair_of_row,

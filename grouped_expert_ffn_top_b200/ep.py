@@ -23,9 +23,12 @@ order with the library's permute kernel used as a row scatter (k = 1), and
 the inverse is its permute backward used as a row gather.
 
 The exchanges are torch.distributed all-to-alls (NCCL on GPUs): the split
-sizes have to be known on the host, so each exchange of rows follows one
-small device-to-host copy of the counts. The local steps run in `ops`, the
-library's kernels through the C ABI (`KernelOps`).
+sizes have to be known on the host, so the forward makes one small
+device-to-host copy of the counts (the received counts and this rank's send
+splits together); the backward reuses those splits. The regroup map and the
+local experts' offsets are built on the device from the received counts
+(moe_ep_regroup). The local steps run in `ops`, the library's kernels through
+the C ABI (`KernelOps`).
 """
 from __future__ import annotations
 
@@ -36,6 +39,10 @@ import torch
 import torch.distributed as dist
 
 from . import native as N
+
+
+def _no_mark(name: str) -> None:
+    pass
 
 
 class KernelOps:
@@ -51,6 +58,11 @@ class KernelOps:
 
     def permute(self, x, row_of_pair, k):
         return N.moe_permute(x, row_of_pair, k)
+
+    def regroup(self, recv_dev, recv_host):
+        """Row map and local offsets of the received rows, built on the
+        device from the counts there (moe_ep_regroup)."""
+        return N.moe_ep_regroup(recv_dev, int(recv_host.sum()))
 
     def gather_rows(self, src, rows_of):
         """out[i] = src[rows_of[i]] (the permute backward with k = 1)."""
@@ -80,7 +92,8 @@ class KernelOps:
 
 
 def regroup_map(recv_counts: np.ndarray) -> np.ndarray:
-    """Destination of every received row. recv_counts[s, e] rows for local
+    """The host form of moe_ep_regroup's row map (for ops that keep their
+    tensors on the host). Destination of every received row. recv_counts[s, e] rows for local
     expert e arrive from rank s, sources in rank order and, within a source,
     experts in order; row q of block (s, e) goes to
         sum_{e' < e} sum_s' recv_counts[s', e'] + sum_{s' < s} recv_counts[s', e] + q,
@@ -138,46 +151,67 @@ class EPMoELayer:
                                    group=self.group)
         return out
 
-    def _exchange_counts(self, counts: torch.Tensor) -> np.ndarray:
+    def _exchange_counts(self, counts: torch.Tensor, group_counts: torch.Tensor):
+        """All-to-all of the per-expert counts; returns the received counts on
+        the device [G, El], and on the host (with this rank's own send splits)
+        from one device-to-host copy: the split sizes of the row all-to-alls
+        must be known on the host."""
         recv = torch.empty_like(counts)
         if not self.dist:
             recv.copy_(counts)
         else:
             dist.all_to_all_single(recv, counts, group=self.group)
-        return recv.cpu().numpy().reshape(self.G, self.El)
+        host = torch.cat([recv, group_counts.to(recv.dtype)]).cpu().numpy()
+        n = self.G * self.El
+        return recv.view(self.G, self.El), host[:n].reshape(self.G, self.El), [int(v) for v in host[n:]]
 
     # -- forward / backward -------------------------------------------------
 
-    def forward(self, x: torch.Tensor) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, mark=None) -> torch.Tensor:
+        """Y = layer(x). `mark(name)`, if given, is called after each step
+        (names starting with "a2a" are the exchanges)."""
+        mark = mark or _no_mark
         ops, k, dev = self.ops, self.k, x.device
         T = x.shape[0]
         z = ops.router_logits(x, self.Wr, self.b)
         r = ops.route(z, k, self.G)
         xp = ops.permute(x, r["row_of_pair"], k)
-        recv_counts = self._exchange_counts(r["counts"])
-        send = [int(v) for v in r["group_counts"].cpu().tolist()]
+        mark("route_permute")
+        recv_dev, recv_counts, send = self._exchange_counts(r["counts"], r["group_counts"])
         recv = [int(v) for v in recv_counts.sum(axis=1)]
+        mark("a2a_counts")
         xr = self._a2a_rows(xp, send, recv)
-        m = torch.as_tensor(regroup_map(recv_counts), dtype=torch.int32, device=dev)
-        loc_off = torch.as_tensor(np.concatenate([[0], np.cumsum(recv_counts.sum(axis=0))]),
-                                  dtype=torch.int64, device=dev)
+        mark("a2a_rows_fwd")
+        m, loc_off = ops.regroup(recv_dev, recv_counts)
         xl = ops.permute(xr, m, 1)
         ffn = ops.ffn_fwd(xl, self.Wg, self.Wu, self.Wd, loc_off)
-        yp = self._a2a_rows(ops.gather_rows(ffn["yp"], m), recv, send)
+        yl = ops.gather_rows(ffn["yp"], m)
+        mark("local_ffn_fwd")
+        yp = self._a2a_rows(yl, recv, send)
+        mark("a2a_rows_back")
         Y = ops.combine(yp, r["topk_w"], r["row_of_pair"])
+        mark("combine")
         self.saved = dict(T=T, x=x, z=z, r=r, xp=xp, yp=yp, send=send, recv=recv, m=m, loc_off=loc_off,
                           xl=xl, **{n: ffn[n] for n in ("h1", "h2", "a")})
         return Y
 
-    def backward(self, dY: torch.Tensor, accumulate: bool = True) -> torch.Tensor:
+    def backward(self, dY: torch.Tensor, accumulate: bool = True, mark=None) -> torch.Tensor:
+        mark = mark or _no_mark
         ops, k, s = self.ops, self.k, self.saved
         r, g = s["r"], self.grads
         dyp, dg = ops.combine_bwd(dY, s["yp"], r["topk_w"], r["row_of_pair"])
         dlogits = ops.route_bwd(dg, r["topk_w"], r["topk_idx"], self.E)
-        dyl = ops.permute(self._a2a_rows(dyp, s["send"], s["recv"]), s["m"], 1)
+        mark("combine_route_bwd")
+        dyr = self._a2a_rows(dyp, s["send"], s["recv"])
+        mark("a2a_rows_bwd")
+        dyl = ops.permute(dyr, s["m"], 1)
         dxl = ops.ffn_bwd(s["xl"], self.Wg, self.Wu, self.Wd, s["h1"], s["h2"], s["a"], dyl, s["loc_off"],
                           g["dWg"], g["dWu"], g["dWd"], accumulate)
-        dxp = self._a2a_rows(ops.gather_rows(dxl, s["m"]), s["recv"], s["send"])
+        dxr = ops.gather_rows(dxl, s["m"])
+        mark("local_ffn_bwd")
+        dxp = self._a2a_rows(dxr, s["recv"], s["send"])
+        mark("a2a_rows_bwd_back")
         dX = ops.permute_bwd(dxp, r["row_of_pair"], dlogits, self.Wr, r["topk_idx"], s["T"], k)
         ops.router_bwd(s["xp"], dlogits, r["pair_of_row"], r["offsets"], k, g["dWr"], g["db"], accumulate)
+        mark("permute_router_bwd")
         return dX

@@ -65,6 +65,7 @@ _SIGNATURES = {
     "moe_grouped_ffn_dgrad": ([_p] * 6 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
     "moe_grouped_ffn_wgrad": ([_p] * 5 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _i, _p, _sz, _p], _i),
     "moe_permute_bwd": ([_p, _p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p], _i),
+    "moe_ep_regroup": ([_p, _i, _i, _p, _p, _p], _i),
     "moe_router_bwd_workspace_bytes": ([_i64, _i, _i], _sz),
     "moe_router_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _i, _p, _p, _i, _p, _sz, _p], _i),
     "moe_aux_loss_workspace_bytes": ([_i64, _i], _sz),
@@ -438,6 +439,20 @@ def moe_permute_bwd(dxp, row_of_pair, dlogits, Wr, topk_idx, T: int, k: int, dX=
     _check(lib().moe_permute_bwd(_ptr(dxp), _ptr(row_of_pair), _ptr(dlogits), _ptr(Wr), _ptr(topk_idx),
                                  _dt(dxp), T, d, E, k, _ptr(dX), _stream(stream)), "moe_permute_bwd")
     return dX
+
+
+def moe_ep_regroup(recv_counts, rows: int, stream=None):
+    """Row map [rows] int32 and local offsets [El+1] int64 of the received
+    rows (recv_counts [G, El] int32 on the device; rows = its sum, which the
+    caller knows from its host copy of the counts)."""
+    _contig(recv_counts)
+    G, El = recv_counts.shape
+    dev = recv_counts.device
+    row_map = torch.empty(max(rows, 1), dtype=torch.int32, device=dev)
+    local_offsets = torch.empty(El + 1, dtype=torch.int64, device=dev)
+    _check(lib().moe_ep_regroup(_ptr(recv_counts), G, El, _ptr(row_map), _ptr(local_offsets),
+                                _stream(stream)), "moe_ep_regroup")
+    return row_map[:rows], local_offsets
 
 
 def moe_router_bwd_workspace_bytes(rows, d, E) -> int:

@@ -365,6 +365,27 @@ MOE_API int moe_permute_bwd(const void* dxp, const int32_t* row_of_pair, const f
                     const void* Wr, const int32_t* topk_idx, int dtype, int64_t T, int d,
                     int E, int k, void* dX, cudaStream_t stream);
 
+/* Expert-parallel regroup (expert communication groups, ART issue #917
+ * "Support combined expert and data parallelism in TrainerRank", Desired
+ * behavior; EP token dispatch, leap-finetune PR #26 Summary). After the
+ * dispatch all-to-all, a rank holds rows from G source ranks, each source's
+ * rows grouped by this rank's El local experts in expert order (the R4 group
+ * layout of moe_route on the sender). This call builds, on the device, the
+ * map that sorts them by (local expert, source rank, arrival):
+ *   recv_counts   [G, El] int32  rows received from source s for local expert e
+ *   row_map       [sum recv_counts] int32 output: received row i goes to
+ *                 row row_map[i] (a scatter for moe_permute with k = 1; its
+ *                 inverse gather is moe_permute_bwd with k = 1)
+ *   local_offsets [El+1] int64 output: local expert e owns sorted rows
+ *                 [local_offsets[e], local_offsets[e+1]) (the expert_offsets
+ *                 of the grouped FFN calls on this rank)
+ * row_map must hold sum(recv_counts) entries (at least one); the counts are
+ * read on the device only, so no host synchronisation is needed.
+ * Errors: INVALID_ARG (null pointer, G or El < 1), UNSUPPORTED
+ * (G * El > MOE_MAX_EXPERTS). */
+MOE_API int moe_ep_regroup(const int32_t* recv_counts, int G, int El, int32_t* row_map,
+                           int64_t* local_offsets, cudaStream_t stream);
+
 /* Workspace of moe_router_bwd, in bytes (rows = T*k). */
 MOE_API size_t moe_router_bwd_workspace_bytes(int64_t rows, int d, int E);
 

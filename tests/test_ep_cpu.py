@@ -58,6 +58,12 @@ class OracleOps:
         por[rop] = np.arange(rop.size, dtype=rop.dtype)
         return _t(self.o.permute(x.numpy(), por, k)) if rop.size else x.new_empty((0, x.shape[1]))
 
+    def regroup(self, recv_dev, recv_host):
+        """The regroup map and local offsets on the host (regroup_map)."""
+        m = torch.as_tensor(regroup_map(recv_host), dtype=torch.int64)
+        off = torch.as_tensor(np.concatenate([[0], np.cumsum(recv_host.sum(axis=0))]), dtype=torch.int64)
+        return m, off
+
     def gather_rows(self, src, rows_of):
         if rows_of.numel() == 0:
             return src.new_empty((0, src.shape[1]))

@@ -81,3 +81,28 @@ def test_one_rank_expert_parallel_layer_is_the_plain_layer():
 
 def test_one_rank_nccl_expert_parallel_layer_is_the_plain_layer():
     _compare(with_group=True)
+
+
+@pytest.mark.parametrize("G,El,zero", [(1, 8, False), (2, 4, False), (4, 16, False), (8, 2, False),
+                                       (3, 5, False), (16, 64, False), (4, 4, True)])
+def test_device_regroup_map_is_the_stable_sort_by_expert_then_source(G, El, zero):
+    """moe_ep_regroup against an independent definition: received row i
+    (arrival order: source, then local expert, then position) goes to its rank
+    in the order (local expert, source, position)."""
+    rng = np.random.default_rng(G * 100 + El)
+    counts = rng.integers(0, 50, size=(G, El)).astype(np.int32)
+    counts[rng.random((G, El)) < 0.3] = 0
+    if zero:
+        counts[:] = 0
+    rows = int(counts.sum())
+    m, off = N.moe_ep_regroup(torch.as_tensor(counts, device=DEV), rows)
+    torch.cuda.synchronize()
+    flat = counts.reshape(-1)
+    src = np.repeat(np.arange(G * El) // El, flat)
+    exp = np.repeat(np.arange(G * El) % El, flat)
+    pos = np.concatenate([np.arange(c) for c in flat]) if rows else np.zeros(0, np.int64)
+    order = np.lexsort((pos, src, exp))  # primary key: expert, then source, then position
+    dest = np.empty(rows, np.int64)
+    dest[order] = np.arange(rows)
+    assert np.array_equal(to_np(m).astype(np.int64), dest)
+    assert np.array_equal(to_np(off), np.concatenate([[0], np.cumsum(counts.sum(axis=0))]))
