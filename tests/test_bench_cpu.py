@@ -49,3 +49,51 @@ def test_workload_config_names_the_shape():
     assert c["workload"] == "fine_fwdbwd_32k"
     assert (c["tokens_per_gpu"], c["d_model"], c["experts"], c["top_k"], c["ffn"]) == (32768, 2048, 64, 8, 1408)
     assert "l2" in c
+
+
+def test_workload_config_of_the_sweep_names_its_microbatches():
+    w = workloads.WORKLOADS["uneven_sweep"]
+    c = bench.workload_config(w)
+    assert c["microbatches"] == [32768, 9000, 1, 0] and c["tokens_per_gpu"] == 41769
+    assert "add to them" in c["grads"]
+    assert bench.metric_of(w) == "MoE layer fwd+bwd tokens/s"
+    assert bench.metric_of(workloads.WORKLOADS["dense_fwd"]) == "MoE layer fwd tokens/s"
+
+
+def test_expert_parallel_ranks_get_uneven_work_and_one_empty_rank():
+    assert bench.ep_tokens(32768, 1) == [32768]
+    assert bench.ep_tokens(32768, 2) == [32768, 16384]
+    assert bench.ep_tokens(32768, 4) == [32768, 16384, 8192, 0]
+
+
+def _run_bench(args, env_extra=None, timeout=600):
+    import os
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    env.update(env_extra or {})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    return subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, capture_output=True,
+                          text=True, timeout=timeout, env=env, cwd=root)
+
+
+def test_gpus_two_without_a_launcher_starts_two_ranks():
+    """`--gpus 2` re-executes bench.py under torch.distributed.run with two
+    ranks; on the reference arm rank 0 times the oracle and reports n_gpus 2,
+    the other rank exits without work."""
+    import json
+    r = _run_bench(["--impl", "reference", "--gpus", "2", "--workload", "tiny_fp32", "--steps", "3",
+                    "--warmup", "3"])
+    assert r.returncode == 0, r.stdout + r.stderr
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["impl"] == "reference" and line["ranks_working"] == 1
+    assert line["config"]["workload"] == "tiny_fp32" and line["value"] > 0
+
+
+def test_gpus_must_match_the_launchers_world_size():
+    r = _run_bench(["--impl", "reference", "--gpus", "2", "--workload", "tiny_fp32"],
+                   env_extra={"WORLD_SIZE": "1", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode != 0
+    assert "WORLD_SIZE=1" in r.stderr
