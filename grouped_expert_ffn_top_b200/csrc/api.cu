@@ -60,7 +60,9 @@ int check_ffn(const char* fn, int dtype, int64_t rows, int E, int d, int f) {
                 static_cast<long long>(rows), E, d, f);
   if (E > MOE_MAX_EXPERTS) return fail(MOE_ERR_UNSUPPORTED, "%s: E=%d > %d", fn, E, MOE_MAX_EXPERTS);
   if (rows >= (int64_t(1) << 31)) return fail(MOE_ERR_UNSUPPORTED, "%s: rows exceed int32", fn);
-  const int q = dtype == MOE_BF16 ? 64 : 4;
+  // bf16: 16-byte rows for TMA (the last K block and the last column tile
+  // past d or f are zero-filled and masked); fp32 (CUDA cores): 16-byte vectors
+  const int q = dtype == MOE_BF16 ? 8 : 4;
   if (d % q != 0 || f % q != 0)
     return fail(MOE_ERR_UNSUPPORTED, "%s: d=%d and f=%d must be multiples of %d for this dtype",
                 fn, d, f, q);
@@ -486,6 +488,7 @@ static int ffn_bwd_impl(const char* fn, const void* xp, const moe::RowGather& g,
   moe::FfnBwdArgs args{xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, rows, E, d, f, dxp,
                        dWg, dWu, dWd, base + moe::kWsHeader, base + moe::kWsHeader + h,
                        static_cast<unsigned*>(ws), accumulate, g};
+  args.maps = base + moe::kWsHeader + 2 * h;  // the weight-gradient kernel's expert maps
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
                                     : moe::launch_ffn_dgrad_f32(args, stream);
   if (e == cudaSuccess) {
@@ -493,7 +496,7 @@ static int ffn_bwd_impl(const char* fn, const void* xp, const moe::RowGather& g,
     e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
                           : moe::launch_ffn_wgrad_f32(args, stream);
   }
-  return launched(cuda_status(e, fn), 1);
+  return launched(cuda_status(e, fn), dtype == MOE_BF16 ? 2 : 1);
 }
 
 static int ffn_wgrad_impl(const char* fn, const void* xp, const moe::RowGather& g, const void* a,
@@ -517,13 +520,16 @@ static int ffn_wgrad_impl(const char* fn, const void* xp, const moe::RowGather& 
   const void* ptrs[] = {xp, a, dyp, dh1, dh2, dWg, dWu, dWd, ws};
   for (const void* q : ptrs)
     if (!aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "%s: 16-byte alignment", fn);
-  if (ws_bytes < moe::kWsHeader) return fail(MOE_ERR_WORKSPACE, "%s: workspace", fn);
+  if (ws_bytes < moe_grouped_ffn_wgrad_workspace_bytes(E, dtype))
+    return fail(MOE_ERR_WORKSPACE, "%s: workspace needs %zu bytes (got %zu)", fn,
+                moe_grouped_ffn_wgrad_workspace_bytes(E, dtype), ws_bytes);
   moe::FfnBwdArgs args{xp, nullptr, nullptr, nullptr, nullptr, nullptr, a, dyp, expert_offsets,
                        rows, E, d, f, nullptr, dWg, dWu, dWd, const_cast<void*>(dh1),
                        const_cast<void*>(dh2), static_cast<unsigned*>(ws), accumulate, g};
+  args.maps = static_cast<uint8_t*>(ws) + moe::kWsHeader;
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
                                     : moe::launch_ffn_wgrad_f32(args, stream);
-  return launched(cuda_status(e, fn), 1);
+  return launched(cuda_status(e, fn), dtype == MOE_BF16 ? 2 : 1);
 }
 
 static moe::RowGather row_gather(const int32_t* pair_of_row, int64_t T, int k) {
@@ -573,10 +579,15 @@ int moe_grouped_ffn_recompute_gather(const void* x, const int32_t* pair_of_row, 
 }
 
 size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype) {
-  (void)E; (void)d;
-  if (rows < 0 || f < 1 || !dtype_ok(dtype)) return 0;
+  (void)d;
+  if (rows < 0 || E < 1 || f < 1 || !dtype_ok(dtype)) return 0;
   const size_t h = align256(static_cast<size_t>(rows) * f * elem_bytes(dtype));
-  return moe::kWsHeader + 2 * h;
+  return moe::kWsHeader + 2 * h + (dtype == MOE_BF16 ? align256(moe::wgrad_maps_bytes(E)) : 0);
+}
+
+size_t moe_grouped_ffn_wgrad_workspace_bytes(int E, int dtype) {
+  if (E < 1 || !dtype_ok(dtype)) return 0;
+  return moe::kWsHeader + (dtype == MOE_BF16 ? align256(moe::wgrad_maps_bytes(E)) : 0);
 }
 
 int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,

@@ -43,6 +43,14 @@ struct Roles {
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
 };
 constexpr int kMaxE = MOE_MAX_EXPERTS;
+// Grouped raster of one expert's tiles: row tiles (M-ragged kinds) or M tiles
+// (wgrad) are taken in groups of this many, and within a group the column
+// tiles advance slowest. The persistent CTAs work on consecutive tiles at any
+// moment, so the tiles in flight together share a few row tiles and a few
+// column tiles: their operands stay in L2 across the group instead of being
+// streamed again from HBM for every row tile.
+constexpr int kRasterRows = 16;
+constexpr int kRasterM = 8;
 constexpr long long kWaitLimit = 2000000000LL;  // about one second of SM cycles
 constexpr uint32_t kTmemCols = 512;
 
@@ -72,6 +80,10 @@ struct Params {
   float* w2;
   unsigned* err;
   int accumulate;  // wgrad: 1 adds to dW, 0 writes it (zero tiles for experts with no rows)
+  // wgrad: five tensor maps per expert (xp, a, dh1, dh2, dyp), each based at
+  // the expert's first row and bounded by its row count, so TMA reads the
+  // rows past the expert's end as zero (built by wgrad_expert_maps_kernel)
+  const CUtensorMap* xmaps;
   // Gathered A rows (kernels instantiated with GATHER): dispatch row r of the
   // expert input is row grow[r] / gk of x [gT, d], the token whose copy xp[r]
   // would be; rows at or past `grows` (the tile's rows past the last expert)
@@ -138,6 +150,16 @@ struct TileInfo {
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Tile `local` of an R x C grid in groups of G rows: (row, column) with the
+// row fastest inside a group of min(G, R - first row) rows.
+__device__ __forceinline__ void raster(int local, int R, int C, int G, int& row, int& col) {
+  const int g = local / (G * C);
+  const int rem = local - g * G * C;
+  const int rg = min(G, R - g * G);
+  col = rem / rg;
+  row = g * G + rem % rg;
+}
+
 // Tiles of an expert with `cnt` rows. Writing weight gradients (accumulate
 // = 0), an expert with no rows still has its tiles: they store zeros.
 template <int KIND, int BN, bool PAIR>
@@ -150,11 +172,15 @@ __device__ __forceinline__ int tiles_of_expert(int cnt, int d, int f, int accumu
   return ceil_div(cnt, Tr::TM) * ceil_div(n_extent, Tr::NTILE);
 }
 
+// K blocks of a tile. When d or f is not a multiple of 64 the last block of
+// each K range runs past it: TMA reads those columns (and the weight rows past
+// the expert's matrix, through the 3D weight maps) as zero, so they add
+// nothing.
 template <int KIND, int BN>
 __device__ __forceinline__ int num_kblocks(const TileInfo& ti, int d, int f) {
-  if (KIND == kFwdGateUp || KIND == kBwdDgradDown) return d / BK;
-  if (KIND == kFwdDown) return f / BK;
-  if (KIND == kBwdDgradGateUp) return 2 * (f / BK);
+  if (KIND == kFwdGateUp || KIND == kBwdDgradDown) return ceil_div(d, BK);
+  if (KIND == kFwdDown) return ceil_div(f, BK);
+  if (KIND == kBwdDgradGateUp) return 2 * ceil_div(f, BK);
   return ceil_div(ti.rows, BK);  // wgrad: ragged K
 }
 
@@ -193,15 +219,19 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d,
       rem = local - 2 * t01;
       nt = ceil_div(d, BN);
     }
-    ti.m0 = (rem / nt) * Tr::TM;
-    ti.n0 = (rem % nt) * BN;
+    const int mt = ti.prod < 2 ? ceil_div(d, Tr::TM) : ceil_div(f, Tr::TM);
+    int mi, ni;
+    raster(rem, mt, nt, kRasterM, mi, ni);
+    ti.m0 = mi * Tr::TM;
+    ti.n0 = ni * BN;
     ti.row0 = base;
     ti.rows = cnt;
   } else {
     const int n_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? f : d;
     const int nt = ceil_div(n_extent, Tr::NTILE);
-    const int mi = local / nt;
-    ti.n0 = (local % nt) * Tr::NTILE;
+    int mi, ni;
+    raster(local, ceil_div(cnt, Tr::TM), nt, kRasterRows, mi, ni);
+    ti.n0 = ni * Tr::NTILE;
     ti.row0 = base + mi * Tr::TM;
     ti.rows = min(Tr::TM, cnt - mi * Tr::TM);
     ti.m0 = 0;
@@ -210,41 +240,47 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d,
   return ti;
 }
 
+// The weight-gradient tile's operand maps (the expert's own, see Params::xmaps):
+// A = xp (dWg, dWu) or a (dWd); B = dh1, dh2 or dyp.
+__device__ __forceinline__ const CUtensorMap* wgrad_map_a(const Params& p, const TileInfo& ti) {
+  return p.xmaps + 5 * ti.e + (ti.prod == 2 ? 1 : 0);
+}
+__device__ __forceinline__ const CUtensorMap* wgrad_map_b(const Params& p, const TileInfo& ti) {
+  return p.xmaps + 5 * ti.e + 2 + ti.prod;
+}
+
 // TMA loads of k block `kb` of tile `ti` into one pipeline stage.
 template <int KIND, int BN>
-__device__ __forceinline__ void issue_loads(const Maps& m, const TileInfo& ti, int kb, int d,
-                                            int f, uint8_t* a_dst, uint8_t* b_dst,
+__device__ __forceinline__ void issue_loads(const Maps& m, const Params& p, const TileInfo& ti, int kb,
+                                            int d, int f, uint8_t* a_dst, uint8_t* b_dst,
                                             uint64_t* bar) {
   const int k0 = kb * BK;
   if (KIND == kFwdGateUp) {
     tma_load_2d(a_dst, &m.a0, bar, k0, ti.row0);
-    const int wrow = ti.e * f + ti.n0;
-    tma_load_2d(b_dst, &m.b0, bar, k0, wrow);
-    tma_load_2d(b_dst + 128 * 128, &m.b1, bar, k0, wrow);
+    tma_load_3d(b_dst, &m.b0, bar, k0, ti.n0, ti.e);
+    tma_load_3d(b_dst + 128 * 128, &m.b1, bar, k0, ti.n0, ti.e);
   } else if (KIND == kFwdDown) {
     tma_load_2d(a_dst, &m.a0, bar, k0, ti.row0);
-    tma_load_2d(b_dst, &m.b0, bar, k0, ti.e * d + ti.n0);
+    tma_load_3d(b_dst, &m.b0, bar, k0, ti.n0, ti.e);
   } else if (KIND == kBwdDgradDown) {
     tma_load_2d(a_dst, &m.a0, bar, k0, ti.row0);
 #pragma unroll
-    for (int j = 0; j < BN / 64; ++j)
-      tma_load_2d(b_dst + j * 8192, &m.b0, bar, ti.n0 + 64 * j, ti.e * d + k0);
+    for (int j = 0; j < BN / 64; ++j) tma_load_3d(b_dst + j * 8192, &m.b0, bar, ti.n0 + 64 * j, k0, ti.e);
   } else if (KIND == kBwdDgradGateUp) {
-    const int half = f / BK;
+    const int half = ceil_div(f, BK);
     const bool second = kb >= half;
     const int kk = (second ? kb - half : kb) * BK;
     tma_load_2d(a_dst, second ? &m.a1 : &m.a0, bar, kk, ti.row0);
 #pragma unroll
     for (int j = 0; j < BN / 64; ++j)
-      tma_load_2d(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + 64 * j, ti.e * f + kk);
-  } else {  // kWgrad: A = xp (dWg, dWu) or a (dWd); B = dh1, dh2 or dyp
-    const CUtensorMap* am = ti.prod == 2 ? &m.a1 : &m.a0;
-    const CUtensorMap* bm = ti.prod == 0 ? &m.b0 : (ti.prod == 1 ? &m.b1 : &m.b2);
-    const int r = ti.row0 + k0;
-    tma_load_2d(a_dst, am, bar, ti.m0, r);
-    tma_load_2d(a_dst + 8192, am, bar, ti.m0 + 64, r);
+      tma_load_3d(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + 64 * j, kk, ti.e);
+  } else {  // kWgrad: A = xp (dWg, dWu) or a (dWd); B = dh1, dh2 or dyp, rows of the expert
+    const CUtensorMap* am = wgrad_map_a(p, ti);
+    const CUtensorMap* bm = wgrad_map_b(p, ti);
+    tma_load_2d(a_dst, am, bar, ti.m0, k0);
+    tma_load_2d(a_dst + 8192, am, bar, ti.m0 + 64, k0);
 #pragma unroll
-    for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, bm, bar, ti.n0 + 64 * j, r);
+    for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, bm, bar, ti.n0 + 64 * j, k0);
   }
 }
 
@@ -253,44 +289,42 @@ __device__ __forceinline__ void issue_loads(const Maps& m, const TileInfo& ti, i
 // on the even CTA's mbarrier at `bar`, a shared::cluster address. With
 // load_a false the A operand is left to the gathered loads.
 template <int KIND, int BN>
-__device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& ti, int kb, int d,
-                                                 int f, int cta, uint8_t* a_dst, uint8_t* b_dst,
-                                                 uint32_t bar, bool load_a = true) {
+__device__ __forceinline__ void issue_loads_pair(const Maps& m, const Params& p, const TileInfo& ti,
+                                                 int kb, int d, int f, int cta, uint8_t* a_dst,
+                                                 uint8_t* b_dst, uint32_t bar, bool load_a = true) {
   const int k0 = kb * BK;
   const int arow = ti.row0 + BM * cta;
   constexpr int HALF = BN / 2;
   if (KIND == kFwdGateUp) {
     if (load_a) tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
-    tma_load_2d_pair(b_dst, cta == 0 ? &m.b0 : &m.b1, bar, k0, ti.e * f + ti.n0);
+    tma_load_3d_pair(b_dst, cta == 0 ? &m.b0 : &m.b1, bar, k0, ti.n0, ti.e);
   } else if (KIND == kFwdDown) {
     tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
-    tma_load_2d_pair(b_dst, &m.b0, bar, k0, ti.e * d + ti.n0 + HALF * cta);
+    tma_load_3d_pair(b_dst, &m.b0, bar, k0, ti.n0 + HALF * cta, ti.e);
   } else if (KIND == kBwdDgradDown) {
     tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
 #pragma unroll
     for (int j = 0; j < HALF / 64; ++j)
-      tma_load_2d_pair(b_dst + j * 8192, &m.b0, bar, ti.n0 + HALF * cta + 64 * j, ti.e * d + k0);
+      tma_load_3d_pair(b_dst + j * 8192, &m.b0, bar, ti.n0 + HALF * cta + 64 * j, k0, ti.e);
   } else if (KIND == kBwdDgradGateUp) {
-    const int half = f / BK;
+    const int half = ceil_div(f, BK);
     const bool second = kb >= half;
     const int kk = (second ? kb - half : kb) * BK;
     tma_load_2d_pair(a_dst, second ? &m.a1 : &m.a0, bar, kk, arow);
 #pragma unroll
     for (int j = 0; j < HALF / 64; ++j)
-      tma_load_2d_pair(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + HALF * cta + 64 * j,
-                       ti.e * f + kk);
+      tma_load_3d_pair(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + HALF * cta + 64 * j, kk, ti.e);
   } else {  // kWgrad: this CTA's 128 values of M and half of N, K rows of the expert
-    const CUtensorMap* am = ti.prod == 2 ? &m.a1 : &m.a0;
-    const CUtensorMap* bm = ti.prod == 0 ? &m.b0 : (ti.prod == 1 ? &m.b1 : &m.b2);
-    const int r = ti.row0 + k0;
+    const CUtensorMap* am = wgrad_map_a(p, ti);
+    const CUtensorMap* bm = wgrad_map_b(p, ti);
     const int mm = ti.m0 + BM * cta;
     if (load_a) {
-      tma_load_2d_pair(a_dst, am, bar, mm, r);
-      tma_load_2d_pair(a_dst + 8192, am, bar, mm + 64, r);
+      tma_load_2d_pair(a_dst, am, bar, mm, k0);
+      tma_load_2d_pair(a_dst + 8192, am, bar, mm + 64, k0);
     }
 #pragma unroll
     for (int j = 0; j < HALF / 64; ++j)
-      tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, r);
+      tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, k0);
   }
 }
 
@@ -315,19 +349,24 @@ __device__ __forceinline__ int token_of_row(const Params& p, int r) {
 //     the epilogue drops: they read column 0 instead.
 template <int KIND>
 __device__ __forceinline__ void gather_a_stage(const Params& p, int lane, uint32_t a_s, int k0,
-                                               int col0, const int (&tok)[4]) {
+                                               int col0, const int (&tok)[4], int valid_rows) {
   const char* xb = reinterpret_cast<const char*>(p.gx);
   const int c = lane & 7;
   if (KIND == kFwdGateUp) {
     const int h = lane >> 3;  // row 4 i + h of iteration i
     const uint32_t d_even = h * 128 + ((c ^ h) << 4);        // (4 i + h) % 8 = h for even i
     const uint32_t d_odd = h * 128 + ((c ^ (h + 4)) << 4);   // and 4 + h for odd i
-    const int64_t cofs = static_cast<int64_t>(k0 + 8 * c) * 2;
+    // K columns at or past d (the last block when d is not a multiple of 64)
+    // are written as zeros without reading x
+    const bool col_in = k0 + 8 * c < p.d;
+    const int64_t cofs = col_in ? static_cast<int64_t>(k0 + 8 * c) * 2 : 0;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int t = __shfl_sync(0xffffffffu, tok[i >> 3], (4 * i + h) & 31);
-      cp_async_16(a_s + i * 512 + ((i & 1) ? d_odd : d_even),
-                  xb + static_cast<int64_t>(t) * p.d * 2 + cofs);
+      const uint32_t dst = a_s + i * 512 + ((i & 1) ? d_odd : d_even);
+      const char* src = xb + static_cast<int64_t>(t) * p.d * 2 + cofs;
+      if (col_in) cp_async_16(dst, src);
+      else cp_async_16_zfill(dst, src, 0u);
     }
   } else {
     const int hh = lane >> 4;        // K row 2 i + hh of iteration i
@@ -336,11 +375,15 @@ __device__ __forceinline__ void gather_a_stage(const Params& p, int lane, uint32
     if (col >= p.d) col = 0;
     const int64_t cofs = static_cast<int64_t>(col) * 2;
     const uint32_t dbase = b * 8192 + hh * 128;
+    // K rows past the expert's end (valid_rows of the block are inside) are
+    // written as zeros, like the TMA-loaded operand's
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int t = __shfl_sync(0xffffffffu, tok[i >> 4], (2 * i + hh) & 31);
       const uint32_t sw = static_cast<uint32_t>(c ^ ((2 * (i & 3) + hh) & 7)) << 4;
-      cp_async_16(a_s + dbase + i * 256 + sw, xb + static_cast<int64_t>(t) * p.d * 2 + cofs);
+      const char* src = xb + static_cast<int64_t>(t) * p.d * 2 + cofs;
+      if (2 * i + hh < valid_rows) cp_async_16(a_s + dbase + i * 256 + sw, src);
+      else cp_async_16_zfill(a_s + dbase + i * 256 + sw, src, 0u);
     }
   }
 }
@@ -408,12 +451,15 @@ __device__ __forceinline__ void epilogue_wgrad(const Params& p, const TileInfo& 
     }
     if (valid && ti.n0 + c < Nn) {
       float* q = out + static_cast<int64_t>(ti.n0 + c) * M;
+      const int nc = min(16, Nn - (ti.n0 + c));  // columns of this group inside the output
       if (p.accumulate) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) red_add_f32(q + static_cast<int64_t>(i) * M, __uint_as_float(u[i]));
+        for (int i = 0; i < 16; ++i)
+          if (i < nc) red_add_f32(q + static_cast<int64_t>(i) * M, __uint_as_float(u[i]));
       } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) q[static_cast<int64_t>(i) * M] = __uint_as_float(u[i]);
+        for (int i = 0; i < 16; ++i)
+          if (i < nc) q[static_cast<int64_t>(i) * M] = __uint_as_float(u[i]);
       }
     }
   }
@@ -493,12 +539,15 @@ __device__ __forceinline__ void epilogue_tma(const Params& p, const Maps& maps, 
       }
       ebuf ^= 1;
     } else if (lane < valid) {
+      // the chunk's columns inside the output (a multiple of 8)
+      const int ncol = min(32, ncols - (ti.n0 + c));
 #pragma unroll
       for (int t = 0; t < NT; ++t) {
         if (!optr[t]) continue;
         bf16* dst = optr[t] + row * ncols + ti.n0 + c;
-        store16_bf16(dst, o[t]);
-        store16_bf16(dst + 16, o[t] + 16);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (8 * j < ncol) *reinterpret_cast<uint4*>(dst + 8 * j) = pack8_bf16(o[t] + 8 * j);
       }
     }
   }
@@ -523,7 +572,7 @@ __device__ __forceinline__ bool epilogue_swiglu_bwd(const Params& p, const Maps&
   constexpr uint32_t BOX = 32 * 32 * 2;
   const int valid = min(32, ti.rows - rbase);
   if (valid <= 0) return true;
-  const int nch = min(BN, p.f - ti.n0) / 32;
+  const int nch = ceil_div(min(BN, p.f - ti.n0), 32);  // the last chunk may run past f
   const int y = ti.row0 + rbase;
   const int64_t row = static_cast<int64_t>(y) + lane;
   // buffer pair b: h1 (then dh1) at sbuf + 2 b BOX, h2 (then dh2) after it
@@ -586,10 +635,13 @@ __device__ __forceinline__ bool epilogue_swiglu_bwd(const Params& p, const Maps&
     } else {
       if (lane < valid) {
         const int64_t off = row * p.f + ti.n0 + 32 * ch;
-        store16_bf16(p.o0 + off, dh1);
-        store16_bf16(p.o0 + off + 16, dh1 + 16);
-        store16_bf16(p.o1 + off, dh2);
-        store16_bf16(p.o1 + off + 16, dh2 + 16);
+        const int ncol = min(32, p.f - (ti.n0 + 32 * ch));  // a multiple of 8
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (8 * j < ncol) {
+            *reinterpret_cast<uint4*>(p.o0 + off + 8 * j) = pack8_bf16(dh1 + 8 * j);
+            *reinterpret_cast<uint4*>(p.o1 + off + 8 * j) = pack8_bf16(dh2 + 8 * j);
+          }
       }
       __syncwarp();
     }
@@ -761,9 +813,16 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     uint32_t issued_mask = 0, issued_par = 0;  // last load issued on full[s], and its phase
     // loads of both CTAs of a pair complete on the even CTA's full barriers
     const uint32_t full_leader = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
+    int map_key = -1;  // wgrad: expert and product whose tensor maps this thread last used
     for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step) {
       const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
+      if (KIND == kWgrad && lane == 0 && nk > 0 && 3 * ti.e + ti.prod != map_key) {
+        // the expert's maps were written by the preceding launch
+        tensormap_acquire(wgrad_map_a(p, ti));
+        tensormap_acquire(wgrad_map_b(p, ti));
+        map_key = 3 * ti.e + ti.prod;
+      }
       // gathered A: the tokens of this lane's rows (gate/up: rows l + 32 q of
       // the CTA's 128, the same for all k blocks of the tile; wgrad: K rows
       // l + 32 q of the k block, read one block ahead so that the loads'
@@ -785,14 +844,15 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         if (lane == 0) {
           if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
           if (PAIR) {
-            issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst, full_addr, !gath);
+            issue_loads_pair<KIND, BN>(maps, p, ti, kb, d, f, cta, a_dst, b_dst, full_addr, !gath);
           } else {
-            issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
+            issue_loads<KIND, BN>(maps, p, ti, kb, d, f, a_dst, b_dst, &full[stage]);
           }
         }
         if (GATHER) {
           if (gath) {
-            gather_a_stage<KIND>(p, lane, smem_u32(a_dst), kb * BK, ti.m0 + BM * cta, tok);
+            gather_a_stage<KIND>(p, lane, smem_u32(a_dst), kb * BK, ti.m0 + BM * cta, tok,
+                                 ti.rows - kb * BK);
             if (KIND == kWgrad && kb + 1 < nk) {
               tok[0] = token_of_row(p, ti.row0 + (kb + 1) * BK + lane);
               tok[1] = token_of_row(p, ti.row0 + (kb + 1) * BK + lane + 32);
@@ -860,10 +920,10 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         }
       }
       if (KIND == kWgrad && ok && nfull < nk) {
-        // ragged-K tail block: rows past the expert's end belong to the next
-        // expert (or lie past the tensor). Only the 16-row MMA steps that
-        // hold valid rows run, and the invalid rows inside the last of them
-        // are zeroed in both operands first.
+        // ragged-K tail block: the expert's own tensor maps end at its last
+        // row, so TMA has filled the rows past it with zeros in both
+        // operands (the gathered A rows likewise); only the 16-row MMA steps
+        // that hold valid rows run.
         const int kb = nfull;
         if (!wait_stage<GATHER>(full, gfull, stage, phase, s_abort)) {
           ok = false;
@@ -871,26 +931,6 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
           tc_fence_after();
           const int valid = ti.rows - kb * BK;
           const int ksteps = (valid + 15) / 16;
-          const int zrows = ksteps * 16 - valid;
-          if (zrows > 0) {
-            // each 64-column box holds one 128-byte row per K row, so the rows
-            // to clear are one contiguous range per box; a pair's MMA also
-            // reads the odd CTA's stage, which this warp clears through
-            // distributed shared memory
-            const uint32_t a_st = smem_u32(sA + stage * Tr::A_BYTES);
-            const uint32_t b_st = smem_u32(sB + stage * Tr::B_BYTES);
-            const int chunks = zrows * 8;  // 16-byte chunks per box
-            constexpr int kBoxes = 2 + static_cast<int>(Tr::B_BYTES / 8192);
-            for (int peer = 0; peer < (PAIR ? 2 : 1); ++peer) {
-              for (int box = 0; box < kBoxes; ++box) {
-                uint32_t base = (box < 2 ? a_st + box * 8192 : b_st + (box - 2) * 8192) + valid * 128;
-                if (PAIR) base = mapa_shared(base, static_cast<uint32_t>(peer));
-                for (int c = lane; c < chunks; c += 32) st_cluster_zero16(base + 16u * c);
-              }
-            }
-            if (PAIR) fence_proxy_async_cluster();
-            else fence_proxy_async_smem();
-          }
           __syncwarp();
           if (lane == 0) {
             const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
@@ -951,7 +991,6 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   } else if (warp >= 2) {
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;
-    const int r = BM * cta + q * 32 + lane;  // row of the tile
     // with eight epilogue warps each handles half of the columns
     constexpr int kSplit = Roles<KIND>::kEpiWarps / 4;
     const int c0 = ((warp - 2) >> 2) * ((KIND == kFwdGateUp ? 128 : BN) / kSplit);
@@ -975,7 +1014,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
                                      lphase, s_abort))
           break;
       } else {
-        epilogue_wgrad<BN>(p, ti, tacc, r, c0);
+        epilogue_wgrad<BN>(p, ti, tacc, BM * cta + q * 32 + lane, c0);
       }
       tc_fence_before();
       if (PAIR) mbar_arrive_cluster(tempty_leader + 8u * static_cast<uint32_t>(acc));
@@ -1038,9 +1077,57 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D bf16 tensor [outer, mid, inner] (inner contiguous, dense), box
+// [1, box_mid, box_inner], 128-byte swizzle, out-of-bounds reads as zero: the
+// expert weights, so that rows past one expert's matrix read as zero rather
+// than as the next expert's rows.
+static bool make_map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                      uint32_t box_inner, uint32_t box_mid) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint32_t box[3] = {box_inner, box_mid, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Map of an epilogue's TMA boxes: [rows, cols] bf16, 32 x 32 boxes, 64-byte swizzle.
 static bool make_store_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows) {
   return make_map(m, base, cols, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// The weight-gradient kernel's per-expert tensor maps: map j of expert e is
+// template j with its base moved to the expert's first row and its row count
+// set to the expert's (at least 1; an expert with no rows loads nothing).
+// Templates: 0 xp (x when the rows are gathered: then left as is), 1 a,
+// 2 dh1, 3 dh2, 4 dyp.
+struct WgradMapTemplates {
+  CUtensorMap m[5];
+  uint64_t base[5];   // tensor base addresses
+  uint64_t pitch[5];  // row pitches in bytes
+};
+
+__global__ void __launch_bounds__(128) wgrad_expert_maps_kernel(const __grid_constant__ WgradMapTemplates t,
+                                                                const int64_t* __restrict__ off, int E,
+                                                                int keep_first, CUtensorMap* out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 5 * E) return;
+  const int e = i / 5, j = i % 5;
+  CUtensorMap* m = out + i;
+  const uint4* src = reinterpret_cast<const uint4*>(&t.m[j]);
+  uint4* dst = reinterpret_cast<uint4*>(m);
+#pragma unroll
+  for (int q = 0; q < static_cast<int>(sizeof(CUtensorMap) / 16); ++q) dst[q] = src[q];
+  if (!(keep_first && j == 0)) {
+    const int64_t r0 = off[e];
+    const int64_t n = off[e + 1] - r0;
+    tensormap_replace_address(m, t.base[j] + static_cast<uint64_t>(r0) * t.pitch[j]);
+    tensormap_replace_rows(m, n > 0 ? static_cast<uint32_t>(n) : 1u);
+  }
+  tensormap_release();
 }
 
 static int sm_count() {
@@ -1109,7 +1196,7 @@ cudaError_t launch_ffn_gateup_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   // gathered: the kernel reads x [T, d] itself (the map stays valid but unused)
   if (!(gather ? make_map(&m1.a0, a.xp, d, static_cast<uint64_t>(a.gather.T), d, 64, 1)
                : make_map(&m1.a0, a.xp, d, rows, d, 64, 128)) ||
-      !make_map(&m1.b0, a.Wg, d, E * f, d, 64, 128) || !make_map(&m1.b1, a.Wu, d, E * f, d, 64, 128))
+      !make_map3(&m1.b0, a.Wg, d, f, E, 64, 128) || !make_map3(&m1.b1, a.Wu, d, f, E, 64, 128))
     return cudaErrorInvalidValue;
   p.gx = static_cast<const bf16*>(a.xp);
   p.grow = a.gather.rows;
@@ -1139,7 +1226,7 @@ cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s) {
   p.err = a.err;
   Maps m2{};
   // pairs: each CTA stages 128 of the tile's 256 Wd rows
-  if (!make_map(&m2.a0, a.a, f, rows, f, 64, 128) || !make_map(&m2.b0, a.Wd, f, E * d, f, 64, 128))
+  if (!make_map(&m2.a0, a.a, f, rows, f, 64, 128) || !make_map3(&m2.b0, a.Wd, f, d, E, 64, 128))
     return cudaErrorInvalidValue;
   p.o0 = static_cast<bf16*>(a.yp);
   p.o1 = p.o2 = nullptr;
@@ -1163,7 +1250,7 @@ cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   Params p = bwd_params(a);
   // 1. da = dyp Wd_e, SwiGLU backward in the epilogue -> dh1, dh2
   Maps m1{};
-  if (!make_map(&m1.a0, a.dyp, d, rows, d, 64, 128) || !make_map(&m1.b0, a.Wd, f, E * d, f, 64, 64))
+  if (!make_map(&m1.a0, a.dyp, d, rows, d, 64, 128) || !make_map3(&m1.b0, a.Wd, f, d, E, 64, 64))
     return cudaErrorInvalidValue;
   p.i0 = static_cast<const bf16*>(a.h1);
   p.i1 = static_cast<const bf16*>(a.h2);
@@ -1181,7 +1268,7 @@ cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   // 2. dxp = dh1 Wg_e + dh2 Wu_e
   Maps m2{};
   if (!make_map(&m2.a0, a.dh1, f, rows, f, 64, 128) || !make_map(&m2.a1, a.dh2, f, rows, f, 64, 128) ||
-      !make_map(&m2.b0, a.Wg, d, E * f, d, 64, 64) || !make_map(&m2.b1, a.Wu, d, E * f, d, 64, 64))
+      !make_map3(&m2.b0, a.Wg, d, f, E, 64, 64) || !make_map3(&m2.b1, a.Wu, d, f, E, 64, 64))
     return cudaErrorInvalidValue;
   p.i0 = p.i1 = nullptr;
   p.o0 = static_cast<bf16*>(a.dxp);
@@ -1206,6 +1293,24 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.w1 = a.dWu;
   p.w2 = a.dWd;
   p.accumulate = a.accumulate;
+  // the experts' own maps, bounded by their row counts, in the workspace
+  WgradMapTemplates t;
+  t.m[0] = m3.a0;
+  t.m[1] = m3.a1;
+  t.m[2] = m3.b0;
+  t.m[3] = m3.b1;
+  t.m[4] = m3.b2;
+  const void* bases[5] = {a.xp, a.a, a.dh1, a.dh2, a.dyp};
+  const uint64_t pitches[5] = {d * 2, f * 2, f * 2, f * 2, d * 2};
+  for (int j = 0; j < 5; ++j) {
+    t.base[j] = reinterpret_cast<uint64_t>(bases[j]);
+    t.pitch[j] = pitches[j];
+  }
+  CUtensorMap* xmaps = static_cast<CUtensorMap*>(a.maps);
+  wgrad_expert_maps_kernel<<<(5 * a.E + 127) / 128, 128, 0, s>>>(t, a.offsets, a.E, gather ? 1 : 0, xmaps);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  p.xmaps = xmaps;
   p.gx = static_cast<const bf16*>(a.xp);
   p.grow = a.gather.rows;
   p.gk = a.gather.k;

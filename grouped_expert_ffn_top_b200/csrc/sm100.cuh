@@ -81,6 +81,18 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+// 3D tiled tensor load global -> shared (coordinates x innermost, then y, z),
+// completion counted on `bar` in bytes. Elements outside the tensor read as
+// zero; the full box's bytes are counted either way.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 // TMA tiled store of a 2D box from shared memory to global memory, tracked
 // as part of this thread's current bulk group. Coordinates are element
 // indices (x innermost); parts of the box outside the tensor are not written.
@@ -212,18 +224,6 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// 16 zero bytes at a shared::cluster address (this CTA's or a peer's).
-__device__ __forceinline__ void st_cluster_zero16(uint32_t cluster_addr) {
-  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(cluster_addr), "r"(0u)
-               : "memory");
-}
-
-// Orders this thread's generic-proxy writes to shared::cluster memory before
-// later async-proxy reads of it (a peer CTA's MMA operands).
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
-}
-
 // Arrive on an mbarrier given by its shared::cluster address (possibly in
 // the peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
@@ -240,6 +240,23 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// The 3D form of tma_load_2d_pair.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map,
+                                                 uint32_t bar_cluster_addr, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// 16-byte global -> shared copy of which only the first `src_bytes` (0 or 16)
+// are read; the rest of the 16 bytes is written as zero.
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst_smem, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst_smem), "l"(src), "r"(src_bytes)
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
@@ -274,6 +291,28 @@ __device__ __forceinline__ void mma_commit_pair_multicast(uint64_t* bar, uint16_
       " [%0], %1;" ::"r"(smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
+}
+
+// ---------------------------------------------- tensor maps in global memory
+//
+// A tensor map copied to global memory and changed there (in the generic
+// proxy) becomes visible to TMA after a release fence by the writer and an
+// acquire fence, on that map, by the thread that then issues TMA with it.
+
+__device__ __forceinline__ void tensormap_replace_address(void* map, uint64_t addr) {
+  asm volatile("tensormap.replace.tile.global_address.global.b1024.b64 [%0], %1;" ::"l"(map), "l"(addr)
+               : "memory");
+}
+// The extent of dimension 1 (the rows of a 2D map).
+__device__ __forceinline__ void tensormap_replace_rows(void* map, uint32_t rows) {
+  asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 1, %1;" ::"l"(map), "r"(rows)
+               : "memory");
+}
+__device__ __forceinline__ void tensormap_release() {
+  asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory");
+}
+__device__ __forceinline__ void tensormap_acquire(const void* map) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
 }
 
 // ------------------------------------------------------ UMMA descriptors

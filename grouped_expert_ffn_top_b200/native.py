@@ -61,6 +61,7 @@ _SIGNATURES = {
     "moe_unpermute_combine_bwd": ([_p, _p, _p, _p, _i, _i64, _i, _i, _p, _p, _p], _i),
     "moe_route_bwd": ([_p, _p, _p, _i64, _i, _i, _p, _p], _i),
     "moe_grouped_ffn_bwd_workspace_bytes": ([_i64, _i, _i, _i, _i], _sz),
+    "moe_grouped_ffn_wgrad_workspace_bytes": ([_i, _i], _sz),
     "moe_grouped_ffn_bwd": ([_p] * 8 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _i, _p, _sz, _p], _i),
     "moe_grouped_ffn_dgrad": ([_p] * 6 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _p, _sz, _p], _i),
     "moe_grouped_ffn_wgrad": ([_p] * 5 + [_i, _p, _i64, _i, _i, _i, _p, _p, _p, _i, _p, _sz, _p], _i),
@@ -358,6 +359,10 @@ def moe_router_bwd_dense(x, Wr, dz, dX, dWr, db, accumulate: bool = True, ws=Non
 
 def moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype) -> int:
     return lib().moe_grouped_ffn_bwd_workspace_bytes(rows, E, d, f, dtype)
+
+
+def moe_grouped_ffn_wgrad_workspace_bytes(E, dtype) -> int:
+    return lib().moe_grouped_ffn_wgrad_workspace_bytes(E, dtype)
 
 
 def moe_grouped_ffn_bwd(xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, dWg, dWu, dWd,

@@ -81,6 +81,12 @@ WORKLOADS: Dict[str, Workload] = {
         "fine_fwdbwd_8k", [8192], d=2048, E=64, k=8, f=1408, dtype=BF16, bias="zipf",
         backward=True, ep_groups=4,
         description="the 32k workload's layer on 8192 tokens (kernel profiling: a few GB on the device)"),
+    "sweep_profile": Workload(
+        "sweep_profile", [4096], d=4096, E=2, k=2, f=14336, dtype=BF16,
+        bias=("normal", 1.0), backward=True, ep_groups=1,
+        description="the sweep's layer shapes with 2 experts and 4096 tokens at top-2: every "
+                    "expert gets 4096 rows, the average of the sweep's 32768-token microbatch, "
+                    "an eighth of its work (kernel counter captures: about 3.5 GB on the device)"),
     "uneven_sweep": Workload(
         "uneven_sweep", [32768, 9000, 1, 0], d=4096, E=16, k=2, f=14336, dtype=BF16,
         bias=("normal", 1.0), backward=True, ep_groups=1,

@@ -219,7 +219,7 @@ MOE_API size_t moe_grouped_ffn_fwd_workspace_bytes(int64_t rows, int E, int d, i
  *     then they are not stored, 2 rows * f elements less written, and the
  *     backward rebuilds them with moe_grouped_ffn_recompute; activation
  *     checkpointing)
- * Errors: INVALID_ARG; UNSUPPORTED (bf16 needs d and f multiples of 64,
+ * Errors: INVALID_ARG; UNSUPPORTED (bf16 needs d and f multiples of 8,
  * fp32 needs multiples of 4; E > MOE_MAX_EXPERTS); WORKSPACE. */
 MOE_API int moe_grouped_ffn_fwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,
                         int dtype, const int64_t* expert_offsets, int64_t rows, int E,
@@ -290,7 +290,8 @@ MOE_API int moe_grouped_ffn_recompute_gather(const void* x, const int32_t* pair_
                                              void* h1, void* h2, void* ws, size_t ws_bytes,
                                              cudaStream_t stream);
 
-/* Workspace of moe_grouped_ffn_bwd, in bytes (holds dh1 and dh2). */
+/* Workspace of moe_grouped_ffn_bwd, in bytes (holds dh1, dh2 and, for bf16,
+ * the weight-gradient kernel's per-expert tensor maps). */
 MOE_API size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype);
 
 /* Grouped SwiGLU expert FFN, backward. Per expert e over its rows:
@@ -331,7 +332,15 @@ MOE_API int moe_grouped_ffn_bwd_gather(const void* x, const int32_t* pair_of_row
  * moe_grouped_ffn_wgrad: weight gradients in fp32, added or written as the
  * accumulate flag says (as moe_grouped_ffn_bwd)
  *   dWg_e (+)= dh1^T xp; dWu_e (+)= dh2^T xp; dWd_e (+)= dyp^T a
- * ws needs moe_grouped_ffn_fwd_workspace_bytes() bytes (its error word). */
+ * ws of moe_grouped_ffn_dgrad needs moe_grouped_ffn_fwd_workspace_bytes()
+ * bytes (its error word); ws of moe_grouped_ffn_wgrad needs
+ * moe_grouped_ffn_wgrad_workspace_bytes(E, dtype) bytes. */
+/* Workspace of moe_grouped_ffn_wgrad and moe_grouped_ffn_wgrad_gather, in
+ * bytes: the error word and, for bf16, five 128-byte tensor maps per expert
+ * that the call writes on the device before its GEMM (each expert's operand
+ * rows are read through maps that end at the expert's last row, so the rows
+ * past it read as zero). Calls that overlap on the GPU need their own. */
+MOE_API size_t moe_grouped_ffn_wgrad_workspace_bytes(int E, int dtype);
 MOE_API int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const void* h1,
                                   const void* h2, const void* dyp, int dtype,
                                   const int64_t* expert_offsets, int64_t rows, int E, int d, int f,

@@ -48,6 +48,10 @@ CASES = [
     ("bf16_f_not_256", 520, 320, 6, 2, 448, "bf16", 3, True),
     ("bf16_many_experts", 900, 128, 160, 4, 192, "bf16", 8, True),
     ("bf16_k8", 1500, 256, 64, 8, 192, "bf16", 4, True),
+    # d and f multiples of 8 only: the last K block of the gathered rows is
+    # zero-filled past d, the last column tiles are masked
+    ("bf16_d1000_f1400", 300, 1000, 6, 2, 1400, "bf16", 2, True),
+    ("bf16_d72_f40", 333, 72, 5, 2, 40, "bf16", 1, False),
     ("f32_tiny", 256, 64, 4, 2, 128, "f32", 2, True),
     ("f32_odd", 100, 48, 3, 2, 20, "f32", 1, False),
 ]

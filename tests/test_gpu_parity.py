@@ -103,6 +103,13 @@ LAYER_CASES = [
     ("bf16_f_not_256", 520, 320, 6, 2, 448, "bf16", 3, True),
     # more experts than the deepest GEMM pipeline leaves schedule room for
     ("bf16_many_experts", 900, 128, 160, 4, 192, "bf16", 8, True),
+    # d and f multiples of 8 but not of 64: ragged last K blocks (zero-filled by
+    # TMA, weight rows past an expert's matrix included) and masked last column
+    # tiles, at 8-column granularity (1000 = 15 * 64 + 40, 1400 = 21 * 64 + 56;
+    # f = 40 is less than one K block and one 16-column store group)
+    ("bf16_d1000_f1400", 300, 1000, 6, 2, 1400, "bf16", 2, True),
+    ("bf16_d72_f40", 333, 72, 5, 2, 40, "bf16", 1, False),
+    ("bf16_d136_f1032", 1100, 136, 3, 2, 1032, "bf16", 1, True),
     ("f32_tiny", 256, 64, 4, 2, 128, "f32", 2, True),
     ("f32_odd", 100, 48, 3, 2, 20, "f32", 1, False),
 ]
