@@ -133,6 +133,8 @@ int moe_router_logits(const void* x, const void* Wr, const float* b, int dtype, 
   if (d % 8 != 0) return fail(MOE_ERR_UNSUPPORTED, "moe_router_logits: d=%d not a multiple of 8", d);
   if (T == 0) return MOE_OK;
   if (!x || !Wr || !logits) return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: null pointer");
+  if (!aligned16(x) || !aligned16(Wr))
+    return fail(MOE_ERR_INVALID_ARG, "moe_router_logits: x and Wr must be 16-byte aligned");
   return launched(cuda_status(moe::launch_router_logits(x, Wr, b, dtype, T, d, E, logits, stream),
                               "moe_router_logits"), 1);
 }
@@ -488,7 +490,6 @@ static int ffn_bwd_impl(const char* fn, const void* xp, const moe::RowGather& g,
   moe::FfnBwdArgs args{xp, Wg, Wu, Wd, h1, h2, a, dyp, expert_offsets, rows, E, d, f, dxp,
                        dWg, dWu, dWd, base + moe::kWsHeader, base + moe::kWsHeader + h,
                        static_cast<unsigned*>(ws), accumulate, g};
-  args.maps = base + moe::kWsHeader + 2 * h;  // the weight-gradient kernel's expert maps
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_dgrad_bf16(args, stream)
                                     : moe::launch_ffn_dgrad_f32(args, stream);
   if (e == cudaSuccess) {
@@ -496,7 +497,7 @@ static int ffn_bwd_impl(const char* fn, const void* xp, const moe::RowGather& g,
     e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
                           : moe::launch_ffn_wgrad_f32(args, stream);
   }
-  return launched(cuda_status(e, fn), dtype == MOE_BF16 ? 2 : 1);
+  return launched(cuda_status(e, fn), 1);
 }
 
 static int ffn_wgrad_impl(const char* fn, const void* xp, const moe::RowGather& g, const void* a,
@@ -526,10 +527,9 @@ static int ffn_wgrad_impl(const char* fn, const void* xp, const moe::RowGather& 
   moe::FfnBwdArgs args{xp, nullptr, nullptr, nullptr, nullptr, nullptr, a, dyp, expert_offsets,
                        rows, E, d, f, nullptr, dWg, dWu, dWd, const_cast<void*>(dh1),
                        const_cast<void*>(dh2), static_cast<unsigned*>(ws), accumulate, g};
-  args.maps = static_cast<uint8_t*>(ws) + moe::kWsHeader;
   cudaError_t e = dtype == MOE_BF16 ? moe::launch_ffn_wgrad_bf16(args, stream)
                                     : moe::launch_ffn_wgrad_f32(args, stream);
-  return launched(cuda_status(e, fn), dtype == MOE_BF16 ? 2 : 1);
+  return launched(cuda_status(e, fn), 1);
 }
 
 static moe::RowGather row_gather(const int32_t* pair_of_row, int64_t T, int k) {
@@ -582,12 +582,12 @@ size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, in
   (void)d;
   if (rows < 0 || E < 1 || f < 1 || !dtype_ok(dtype)) return 0;
   const size_t h = align256(static_cast<size_t>(rows) * f * elem_bytes(dtype));
-  return moe::kWsHeader + 2 * h + (dtype == MOE_BF16 ? align256(moe::wgrad_maps_bytes(E)) : 0);
+  return moe::kWsHeader + 2 * h;
 }
 
 size_t moe_grouped_ffn_wgrad_workspace_bytes(int E, int dtype) {
   if (E < 1 || !dtype_ok(dtype)) return 0;
-  return moe::kWsHeader + (dtype == MOE_BF16 ? align256(moe::wgrad_maps_bytes(E)) : 0);
+  return moe::kWsHeader;
 }
 
 int moe_grouped_ffn_bwd(const void* xp, const void* Wg, const void* Wu, const void* Wd,

@@ -80,10 +80,6 @@ struct Params {
   float* w2;
   unsigned* err;
   int accumulate;  // wgrad: 1 adds to dW, 0 writes it (zero tiles for experts with no rows)
-  // wgrad: five tensor maps per expert (xp, a, dh1, dh2, dyp), each based at
-  // the expert's first row and bounded by its row count, so TMA reads the
-  // rows past the expert's end as zero (built by wgrad_expert_maps_kernel)
-  const CUtensorMap* xmaps;
   // Gathered A rows (kernels instantiated with GATHER): dispatch row r of the
   // expert input is row grow[r] / gk of x [gT, d], the token whose copy xp[r]
   // would be; rows at or past `grows` (the tile's rows past the last expert)
@@ -240,19 +236,10 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d,
   return ti;
 }
 
-// The weight-gradient tile's operand maps (the expert's own, see Params::xmaps):
-// A = xp (dWg, dWu) or a (dWd); B = dh1, dh2 or dyp.
-__device__ __forceinline__ const CUtensorMap* wgrad_map_a(const Params& p, const TileInfo& ti) {
-  return p.xmaps + 5 * ti.e + (ti.prod == 2 ? 1 : 0);
-}
-__device__ __forceinline__ const CUtensorMap* wgrad_map_b(const Params& p, const TileInfo& ti) {
-  return p.xmaps + 5 * ti.e + 2 + ti.prod;
-}
-
 // TMA loads of k block `kb` of tile `ti` into one pipeline stage.
 template <int KIND, int BN>
-__device__ __forceinline__ void issue_loads(const Maps& m, const Params& p, const TileInfo& ti, int kb,
-                                            int d, int f, uint8_t* a_dst, uint8_t* b_dst,
+__device__ __forceinline__ void issue_loads(const Maps& m, const TileInfo& ti, int kb, int d,
+                                            int f, uint8_t* a_dst, uint8_t* b_dst,
                                             uint64_t* bar) {
   const int k0 = kb * BK;
   if (KIND == kFwdGateUp) {
@@ -274,13 +261,14 @@ __device__ __forceinline__ void issue_loads(const Maps& m, const Params& p, cons
 #pragma unroll
     for (int j = 0; j < BN / 64; ++j)
       tma_load_3d(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + 64 * j, kk, ti.e);
-  } else {  // kWgrad: A = xp (dWg, dWu) or a (dWd); B = dh1, dh2 or dyp, rows of the expert
-    const CUtensorMap* am = wgrad_map_a(p, ti);
-    const CUtensorMap* bm = wgrad_map_b(p, ti);
-    tma_load_2d(a_dst, am, bar, ti.m0, k0);
-    tma_load_2d(a_dst + 8192, am, bar, ti.m0 + 64, k0);
+  } else {  // kWgrad: A = xp (dWg, dWu) or a (dWd); B = dh1, dh2 or dyp
+    const CUtensorMap* am = ti.prod == 2 ? &m.a1 : &m.a0;
+    const CUtensorMap* bm = ti.prod == 0 ? &m.b0 : (ti.prod == 1 ? &m.b1 : &m.b2);
+    const int r = ti.row0 + k0;
+    tma_load_2d(a_dst, am, bar, ti.m0, r);
+    tma_load_2d(a_dst + 8192, am, bar, ti.m0 + 64, r);
 #pragma unroll
-    for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, bm, bar, ti.n0 + 64 * j, k0);
+    for (int j = 0; j < BN / 64; ++j) tma_load_2d(b_dst + j * 8192, bm, bar, ti.n0 + 64 * j, r);
   }
 }
 
@@ -289,9 +277,9 @@ __device__ __forceinline__ void issue_loads(const Maps& m, const Params& p, cons
 // on the even CTA's mbarrier at `bar`, a shared::cluster address. With
 // load_a false the A operand is left to the gathered loads.
 template <int KIND, int BN>
-__device__ __forceinline__ void issue_loads_pair(const Maps& m, const Params& p, const TileInfo& ti,
-                                                 int kb, int d, int f, int cta, uint8_t* a_dst,
-                                                 uint8_t* b_dst, uint32_t bar, bool load_a = true) {
+__device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& ti, int kb, int d,
+                                                 int f, int cta, uint8_t* a_dst, uint8_t* b_dst,
+                                                 uint32_t bar, bool load_a = true) {
   const int k0 = kb * BK;
   const int arow = ti.row0 + BM * cta;
   constexpr int HALF = BN / 2;
@@ -315,16 +303,17 @@ __device__ __forceinline__ void issue_loads_pair(const Maps& m, const Params& p,
     for (int j = 0; j < HALF / 64; ++j)
       tma_load_3d_pair(b_dst + j * 8192, second ? &m.b1 : &m.b0, bar, ti.n0 + HALF * cta + 64 * j, kk, ti.e);
   } else {  // kWgrad: this CTA's 128 values of M and half of N, K rows of the expert
-    const CUtensorMap* am = wgrad_map_a(p, ti);
-    const CUtensorMap* bm = wgrad_map_b(p, ti);
+    const CUtensorMap* am = ti.prod == 2 ? &m.a1 : &m.a0;
+    const CUtensorMap* bm = ti.prod == 0 ? &m.b0 : (ti.prod == 1 ? &m.b1 : &m.b2);
+    const int r = ti.row0 + k0;
     const int mm = ti.m0 + BM * cta;
     if (load_a) {
-      tma_load_2d_pair(a_dst, am, bar, mm, k0);
-      tma_load_2d_pair(a_dst + 8192, am, bar, mm + 64, k0);
+      tma_load_2d_pair(a_dst, am, bar, mm, r);
+      tma_load_2d_pair(a_dst + 8192, am, bar, mm + 64, r);
     }
 #pragma unroll
     for (int j = 0; j < HALF / 64; ++j)
-      tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, k0);
+      tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, r);
   }
 }
 
@@ -349,7 +338,7 @@ __device__ __forceinline__ int token_of_row(const Params& p, int r) {
 //     the epilogue drops: they read column 0 instead.
 template <int KIND>
 __device__ __forceinline__ void gather_a_stage(const Params& p, int lane, uint32_t a_s, int k0,
-                                               int col0, const int (&tok)[4], int valid_rows) {
+                                               int col0, const int (&tok)[4]) {
   const char* xb = reinterpret_cast<const char*>(p.gx);
   const int c = lane & 7;
   if (KIND == kFwdGateUp) {
@@ -375,15 +364,11 @@ __device__ __forceinline__ void gather_a_stage(const Params& p, int lane, uint32
     if (col >= p.d) col = 0;
     const int64_t cofs = static_cast<int64_t>(col) * 2;
     const uint32_t dbase = b * 8192 + hh * 128;
-    // K rows past the expert's end (valid_rows of the block are inside) are
-    // written as zeros, like the TMA-loaded operand's
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int t = __shfl_sync(0xffffffffu, tok[i >> 4], (2 * i + hh) & 31);
       const uint32_t sw = static_cast<uint32_t>(c ^ ((2 * (i & 3) + hh) & 7)) << 4;
-      const char* src = xb + static_cast<int64_t>(t) * p.d * 2 + cofs;
-      if (2 * i + hh < valid_rows) cp_async_16(a_s + dbase + i * 256 + sw, src);
-      else cp_async_16_zfill(a_s + dbase + i * 256 + sw, src, 0u);
+      cp_async_16(a_s + dbase + i * 256 + sw, xb + static_cast<int64_t>(t) * p.d * 2 + cofs);
     }
   }
 }
@@ -813,16 +798,9 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
     uint32_t issued_mask = 0, issued_par = 0;  // last load issued on full[s], and its phase
     // loads of both CTAs of a pair complete on the even CTA's full barriers
     const uint32_t full_leader = PAIR ? mapa_shared(smem_u32(full), 0) : 0u;
-    int map_key = -1;  // wgrad: expert and product whose tensor maps this thread last used
     for (int tile = first_tile; tile < total && !*s_abort; tile += tile_step) {
       const TileInfo ti = decode_tile<KIND, BN, PAIR>(sched, tile, d, f);
       const int nk = num_kblocks<KIND, BN>(ti, d, f);
-      if (KIND == kWgrad && lane == 0 && nk > 0 && 3 * ti.e + ti.prod != map_key) {
-        // the expert's maps were written by the preceding launch
-        tensormap_acquire(wgrad_map_a(p, ti));
-        tensormap_acquire(wgrad_map_b(p, ti));
-        map_key = 3 * ti.e + ti.prod;
-      }
       // gathered A: the tokens of this lane's rows (gate/up: rows l + 32 q of
       // the CTA's 128, the same for all k blocks of the tile; wgrad: K rows
       // l + 32 q of the k block, read one block ahead so that the loads'
@@ -844,15 +822,14 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         if (lane == 0) {
           if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
           if (PAIR) {
-            issue_loads_pair<KIND, BN>(maps, p, ti, kb, d, f, cta, a_dst, b_dst, full_addr, !gath);
+            issue_loads_pair<KIND, BN>(maps, ti, kb, d, f, cta, a_dst, b_dst, full_addr, !gath);
           } else {
-            issue_loads<KIND, BN>(maps, p, ti, kb, d, f, a_dst, b_dst, &full[stage]);
+            issue_loads<KIND, BN>(maps, ti, kb, d, f, a_dst, b_dst, &full[stage]);
           }
         }
         if (GATHER) {
           if (gath) {
-            gather_a_stage<KIND>(p, lane, smem_u32(a_dst), kb * BK, ti.m0 + BM * cta, tok,
-                                 ti.rows - kb * BK);
+            gather_a_stage<KIND>(p, lane, smem_u32(a_dst), kb * BK, ti.m0 + BM * cta, tok);
             if (KIND == kWgrad && kb + 1 < nk) {
               tok[0] = token_of_row(p, ti.row0 + (kb + 1) * BK + lane);
               tok[1] = token_of_row(p, ti.row0 + (kb + 1) * BK + lane + 32);
@@ -920,10 +897,10 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
         }
       }
       if (KIND == kWgrad && ok && nfull < nk) {
-        // ragged-K tail block: the expert's own tensor maps end at its last
-        // row, so TMA has filled the rows past it with zeros in both
-        // operands (the gathered A rows likewise); only the 16-row MMA steps
-        // that hold valid rows run.
+        // ragged-K tail block: rows past the expert's end belong to the next
+        // expert (or lie past the tensor). Only the 16-row MMA steps that
+        // hold valid rows run, and the invalid rows inside the last of them
+        // are zeroed in both operands first.
         const int kb = nfull;
         if (!wait_stage<GATHER>(full, gfull, stage, phase, s_abort)) {
           ok = false;
@@ -931,6 +908,26 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
           tc_fence_after();
           const int valid = ti.rows - kb * BK;
           const int ksteps = (valid + 15) / 16;
+          const int zrows = ksteps * 16 - valid;
+          if (zrows > 0) {
+            // each 64-column box holds one 128-byte row per K row, so the rows
+            // to clear are one contiguous range per box; a pair's MMA also
+            // reads the odd CTA's stage, which this warp clears through
+            // distributed shared memory
+            const uint32_t a_st = smem_u32(sA + stage * Tr::A_BYTES);
+            const uint32_t b_st = smem_u32(sB + stage * Tr::B_BYTES);
+            const int chunks = zrows * 8;  // 16-byte chunks per box
+            constexpr int kBoxes = 2 + static_cast<int>(Tr::B_BYTES / 8192);
+            for (int peer = 0; peer < (PAIR ? 2 : 1); ++peer) {
+              for (int box = 0; box < kBoxes; ++box) {
+                uint32_t base = (box < 2 ? a_st + box * 8192 : b_st + (box - 2) * 8192) + valid * 128;
+                if (PAIR) base = mapa_shared(base, static_cast<uint32_t>(peer));
+                for (int c = lane; c < chunks; c += 32) st_cluster_zero16(base + 16u * c);
+              }
+            }
+            if (PAIR) fence_proxy_async_cluster();
+            else fence_proxy_async_smem();
+          }
           __syncwarp();
           if (lane == 0) {
             const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
@@ -1099,37 +1096,6 @@ static bool make_store_map(CUtensorMap* m, void* base, uint64_t cols, uint64_t r
   return make_map(m, base, cols, rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// The weight-gradient kernel's per-expert tensor maps: map j of expert e is
-// template j with its base moved to the expert's first row and its row count
-// set to the expert's (at least 1; an expert with no rows loads nothing).
-// Templates: 0 xp (x when the rows are gathered: then left as is), 1 a,
-// 2 dh1, 3 dh2, 4 dyp.
-struct WgradMapTemplates {
-  CUtensorMap m[5];
-  uint64_t base[5];   // tensor base addresses
-  uint64_t pitch[5];  // row pitches in bytes
-};
-
-__global__ void __launch_bounds__(128) wgrad_expert_maps_kernel(const __grid_constant__ WgradMapTemplates t,
-                                                                const int64_t* __restrict__ off, int E,
-                                                                int keep_first, CUtensorMap* out) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= 5 * E) return;
-  const int e = i / 5, j = i % 5;
-  CUtensorMap* m = out + i;
-  const uint4* src = reinterpret_cast<const uint4*>(&t.m[j]);
-  uint4* dst = reinterpret_cast<uint4*>(m);
-#pragma unroll
-  for (int q = 0; q < static_cast<int>(sizeof(CUtensorMap) / 16); ++q) dst[q] = src[q];
-  if (!(keep_first && j == 0)) {
-    const int64_t r0 = off[e];
-    const int64_t n = off[e + 1] - r0;
-    tensormap_replace_address(m, t.base[j] + static_cast<uint64_t>(r0) * t.pitch[j]);
-    tensormap_replace_rows(m, n > 0 ? static_cast<uint32_t>(n) : 1u);
-  }
-  tensormap_release();
-}
-
 static int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -1293,24 +1259,6 @@ cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s) {
   p.w1 = a.dWu;
   p.w2 = a.dWd;
   p.accumulate = a.accumulate;
-  // the experts' own maps, bounded by their row counts, in the workspace
-  WgradMapTemplates t;
-  t.m[0] = m3.a0;
-  t.m[1] = m3.a1;
-  t.m[2] = m3.b0;
-  t.m[3] = m3.b1;
-  t.m[4] = m3.b2;
-  const void* bases[5] = {a.xp, a.a, a.dh1, a.dh2, a.dyp};
-  const uint64_t pitches[5] = {d * 2, f * 2, f * 2, f * 2, d * 2};
-  for (int j = 0; j < 5; ++j) {
-    t.base[j] = reinterpret_cast<uint64_t>(bases[j]);
-    t.pitch[j] = pitches[j];
-  }
-  CUtensorMap* xmaps = static_cast<CUtensorMap*>(a.maps);
-  wgrad_expert_maps_kernel<<<(5 * a.E + 127) / 128, 128, 0, s>>>(t, a.offsets, a.E, gather ? 1 : 0, xmaps);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  p.xmaps = xmaps;
   p.gx = static_cast<const bf16*>(a.xp);
   p.grow = a.gather.rows;
   p.gk = a.gather.k;

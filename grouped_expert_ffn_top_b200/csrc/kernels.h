@@ -77,11 +77,7 @@ struct FfnBwdArgs {
   unsigned* err;
   int accumulate;   // wgrad: 1 adds to dW, 0 writes dW (zero for experts with no rows)
   RowGather gather; // wgrad: xp's rows gathered from x
-  void* maps = nullptr;  // wgrad (bf16): workspace room for wgrad_maps_bytes(E), 64-byte aligned
 };
-// Workspace the bf16 weight-gradient kernel needs for its per-expert tensor
-// maps (5 per expert, 128 bytes each).
-constexpr size_t wgrad_maps_bytes(int E) { return static_cast<size_t>(E) * 5 * 128; }
 
 cudaError_t launch_selftest_wait_timeout(unsigned* err, long long limit, cudaStream_t s);
 
@@ -101,7 +97,7 @@ cudaError_t launch_ffn_fwd_bf16(const FfnFwdArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_gateup_bf16(const FfnFwdArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_gateup_f32(const FfnFwdArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_dgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 2 launches
-cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 2 launches
+cudaError_t launch_ffn_wgrad_bf16(const FfnBwdArgs& a, cudaStream_t s);  // 1 launch
 cudaError_t launch_ffn_fwd_f32(const FfnFwdArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_dgrad_f32(const FfnBwdArgs& a, cudaStream_t s);   // 2 launches
 cudaError_t launch_ffn_wgrad_f32(const FfnBwdArgs& a, cudaStream_t s);   // 1 launch

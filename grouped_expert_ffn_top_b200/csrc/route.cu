@@ -147,14 +147,51 @@ __global__ void __launch_bounds__(NT) router_logits_kernel(const T* __restrict__
   }
 }
 
+// Small batches (T E <= kLogitSmallOutputs): one thread per logit, the
+// fixed-order fma chain over i = 0..d-1 fed by 16-byte loads of its token's
+// x row and its expert's Wr row (four loads in flight). The tiled kernel
+// above stages 64-token tiles through shared memory chunk by chunk, which for
+// a handful of tokens is a chain of load latencies; here the chain is the
+// d dependent FMAs themselves. Same order of operations, same result bits.
+constexpr int64_t kLogitSmallOutputs = 4096;
+
+template <typename T>
+__global__ void __launch_bounds__(128) router_logits_small_kernel(const T* __restrict__ x,
+                                                                  const T* __restrict__ Wr,
+                                                                  const float* __restrict__ b,
+                                                                  int64_t Ttok, int d, int E,
+                                                                  float* __restrict__ z) {
+  constexpr int VE = Vec16<T>::N;
+  const int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (o >= Ttok * E) return;
+  const int64_t t = o / E;
+  const int e = static_cast<int>(o % E);
+  const T* xr = x + t * d;
+  const T* wr = Wr + static_cast<int64_t>(e) * d;
+  float acc = 0.0f;
+#pragma unroll 4
+  for (int i = 0; i < d; i += VE) {
+    const Vec16<T> xv = ld16(xr + i);
+    const Vec16<T> wv = ld16(wr + i);
+#pragma unroll
+    for (int q = 0; q < VE; ++q) acc = __fmaf_rn(xv.get(q), wv.get(q), acc);
+  }
+  z[o] = __fadd_rn(acc, b ? b[e] : 0.0f);
+}
+
 template <typename T>
 static cudaError_t launch_router_logits_t(const T* x, const T* Wr, const float* b, int64_t Ttok,
                                           int d, int E, float* z, cudaStream_t s) {
   const unsigned gx = static_cast<unsigned>((Ttok + kLogitTokens - 1) / kLogitTokens);
-  if (E <= 8) {
+  if (Ttok * E <= kLogitSmallOutputs) {
+    const unsigned blocks = static_cast<unsigned>((Ttok * E + 127) / 128);
+    router_logits_small_kernel<T><<<blocks, 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+  } else if (E <= 8) {
     router_logits_kernel<T, 8, 64><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 16) {
-    router_logits_kernel<T, 16, 128><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    // 8 tokens x 2 experts per thread: twice the FMAs per shared-memory load
+    // of the 8 x 1 tile with 128 threads
+    router_logits_kernel<T, 16, 64><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 32) {
     router_logits_kernel<T, 32, 128><<<dim3(gx, 1), 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else {

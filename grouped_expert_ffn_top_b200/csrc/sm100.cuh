@@ -224,6 +224,18 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// 16 zero bytes at a shared::cluster address (this CTA's or a peer's).
+__device__ __forceinline__ void st_cluster_zero16(uint32_t cluster_addr) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(cluster_addr), "r"(0u)
+               : "memory");
+}
+
+// Orders this thread's generic-proxy writes to shared::cluster memory before
+// later async-proxy reads of it (a peer CTA's MMA operands).
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
 // Arrive on an mbarrier given by its shared::cluster address (possibly in
 // the peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
@@ -291,28 +303,6 @@ __device__ __forceinline__ void mma_commit_pair_multicast(uint64_t* bar, uint16_
       " [%0], %1;" ::"r"(smem_u32(bar)),
       "h"(cta_mask)
       : "memory");
-}
-
-// ---------------------------------------------- tensor maps in global memory
-//
-// A tensor map copied to global memory and changed there (in the generic
-// proxy) becomes visible to TMA after a release fence by the writer and an
-// acquire fence, on that map, by the thread that then issues TMA with it.
-
-__device__ __forceinline__ void tensormap_replace_address(void* map, uint64_t addr) {
-  asm volatile("tensormap.replace.tile.global_address.global.b1024.b64 [%0], %1;" ::"l"(map), "l"(addr)
-               : "memory");
-}
-// The extent of dimension 1 (the rows of a 2D map).
-__device__ __forceinline__ void tensormap_replace_rows(void* map, uint32_t rows) {
-  asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 1, %1;" ::"l"(map), "r"(rows)
-               : "memory");
-}
-__device__ __forceinline__ void tensormap_release() {
-  asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory");
-}
-__device__ __forceinline__ void tensormap_acquire(const void* map) {
-  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(map) : "memory");
 }
 
 // ------------------------------------------------------ UMMA descriptors

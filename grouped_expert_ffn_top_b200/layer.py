@@ -42,12 +42,12 @@ def _no_mark(name: str) -> None:
     pass
 
 
-# Kernels each C call launches (the bf16 path; the fp32 weight gradient is 1).
+# Kernels each C call launches (bf16 and fp32 paths alike).
 LAUNCHES_PER_CALL = {
     "router_logits": 1, "route": 3, "permute": 1, "grouped_ffn_fwd": 2, "unpermute_combine": 1,
-    "unpermute_combine_bwd": 1, "route_bwd": 1, "grouped_ffn_dgrad": 2, "grouped_ffn_wgrad": 2,
+    "unpermute_combine_bwd": 1, "route_bwd": 1, "grouped_ffn_dgrad": 2, "grouped_ffn_wgrad": 1,
     "permute_bwd": 1, "router_bwd": 2, "aux_loss": 2, "aux_loss_bwd": 1, "router_bwd_dense": 3,
-    "grouped_ffn_recompute": 1, "grouped_ffn_fwd_gather": 2, "grouped_ffn_wgrad_gather": 2,
+    "grouped_ffn_recompute": 1, "grouped_ffn_fwd_gather": 2, "grouped_ffn_wgrad_gather": 1,
     "router_bwd_gather": 2, "grouped_ffn_recompute_gather": 1,
 }
 
@@ -113,7 +113,7 @@ class MoELayer:
         self.ws = {
             "route": N._ws(N.moe_route_workspace_bytes(T, E), dev),
             "ffn_fwd": N._ws(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt), dev),
-            # dgrad and recompute use its error word; wgrad also its expert tensor maps
+            # dgrad, wgrad and recompute use its error word
             "ffn_bwd": N._ws(max(N.moe_grouped_ffn_fwd_workspace_bytes(P, E, d, f, self.dt),
                                  N.moe_grouped_ffn_wgrad_workspace_bytes(E, self.dt)), dev),
             "router_bwd": N._ws(N.moe_router_bwd_workspace_bytes(P, d, E), dev),

@@ -119,8 +119,9 @@ MOE_API int moe_get_error(void* ws, cudaStream_t stream);
  *   Wr      [E, d]   dtype      router weight
  *   b       [E]      fp32       router bias (may be NULL: no bias)
  *   logits  [T, E]   fp32       output
- * Errors: INVALID_ARG for null x/Wr/logits with T > 0 or d, E < 1;
- * UNSUPPORTED for E > MOE_MAX_EXPERTS or d not a multiple of 8. */
+ * Errors: INVALID_ARG for null x/Wr/logits with T > 0, d, E < 1, or x, Wr
+ * not 16-byte aligned; UNSUPPORTED for E > MOE_MAX_EXPERTS or d not a
+ * multiple of 8. */
 MOE_API int moe_router_logits(const void* x, const void* Wr, const float* b, int dtype,
                       int64_t T, int d, int E, float* logits, cudaStream_t stream);
 
@@ -290,8 +291,7 @@ MOE_API int moe_grouped_ffn_recompute_gather(const void* x, const int32_t* pair_
                                              void* h1, void* h2, void* ws, size_t ws_bytes,
                                              cudaStream_t stream);
 
-/* Workspace of moe_grouped_ffn_bwd, in bytes (holds dh1, dh2 and, for bf16,
- * the weight-gradient kernel's per-expert tensor maps). */
+/* Workspace of moe_grouped_ffn_bwd, in bytes (holds dh1 and dh2). */
 MOE_API size_t moe_grouped_ffn_bwd_workspace_bytes(int64_t rows, int E, int d, int f, int dtype);
 
 /* Grouped SwiGLU expert FFN, backward. Per expert e over its rows:
@@ -336,10 +336,7 @@ MOE_API int moe_grouped_ffn_bwd_gather(const void* x, const int32_t* pair_of_row
  * bytes (its error word); ws of moe_grouped_ffn_wgrad needs
  * moe_grouped_ffn_wgrad_workspace_bytes(E, dtype) bytes. */
 /* Workspace of moe_grouped_ffn_wgrad and moe_grouped_ffn_wgrad_gather, in
- * bytes: the error word and, for bf16, five 128-byte tensor maps per expert
- * that the call writes on the device before its GEMM (each expert's operand
- * rows are read through maps that end at the expert's last row, so the rows
- * past it read as zero). Calls that overlap on the GPU need their own. */
+ * bytes (its error word). Calls that overlap on the GPU need their own. */
 MOE_API size_t moe_grouped_ffn_wgrad_workspace_bytes(int E, int dtype);
 MOE_API int moe_grouped_ffn_dgrad(const void* Wg, const void* Wu, const void* Wd, const void* h1,
                                   const void* h2, const void* dyp, int dtype,
