@@ -19,8 +19,10 @@ Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 synchronize on both sides, measured with CUDA events on the launching stream;
 the slowest rank's time counts. Per-call CUDA events inside the timed steps
 give each C call's duration. The roofline entry is the grouped weight-gradient
-kernel's launch on the largest microbatch, against the measured bf16 burst
-peak (the sustained fraction is printed beside it).
+kernel's launch on the largest microbatch, against the measured bf16
+sustained peak when the timed region lasts a second or more (the power-capped
+condition that peak was measured in), else the burst peak; both fractions are
+printed beside it.
 The e2e leg repeats the steps through the same C calls with every
 microbatch's x and dY copied from pinned host memory and Y, dX copied back,
 inside the timed region.
@@ -652,13 +654,22 @@ def run_native(args, w):
     rk_ms = mb_ms[(big, rk)]
     rk_flops = algorithmic_work(w, Tb)[0][rk]
     rk_tf = rk_flops / (rk_ms * 1e-3) / 1e12
+    # the peak for the way the kernel was timed: inside a timed region of a
+    # second or more of back-to-back steps the GPU runs under its power cap,
+    # which is where the sustained GEMM peak was measured; a shorter region
+    # runs near the maximum clock (the burst peak)
+    long_region = m["total_ms"] >= 1000.0
+    peak = bf16_sust if long_region else bf16_burst
     line["roofline"] = {
         "kernel": f"{rk} (tcgen05 grouped GEMM{', ragged K' if 'wgrad' in rk else ''}), the launch on "
                   f"the {Tb}-token microbatch",
-        "bound": "tensor", "achieved": round(rk_tf, 1), "peak": bf16_burst, "unit": "TFLOP/s",
-        "frac": round(rk_tf / bf16_burst, 3), "frac_sustained": round(rk_tf / bf16_sust, 3),
+        "bound": "tensor", "achieved": round(rk_tf, 1), "peak": peak, "unit": "TFLOP/s",
+        "frac": round(rk_tf / peak, 3),
+        "frac_burst": round(rk_tf / bf16_burst, 3), "frac_sustained": round(rk_tf / bf16_sust, 3),
         "traffic": ncu_traffic(rk, w.name),
-        "peak_source": f"{peak_src} bf16 burst ({bf16_burst}); sustained {bf16_sust}",
+        "peak_source": (f"{peak_src} bf16 {'sustained' if long_region else 'burst'} "
+                        f"({'timed inside %.1f s of back-to-back steps' % (m['total_ms'] / 1000.0) if long_region else 'timed region under 1 s'}); "
+                        f"burst {bf16_burst}, sustained {bf16_sust}"),
         "algorithmic_flops_per_launch": rk_flops, "ms_per_launch": round(rk_ms, 4)}
     line["kernels"] = kernels
     line["kernels_by_microbatch"] = {
