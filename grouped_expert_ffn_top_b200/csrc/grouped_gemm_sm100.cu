@@ -48,9 +48,17 @@ constexpr int kMaxE = MOE_MAX_EXPERTS;
 // tiles advance slowest. The persistent CTAs work on consecutive tiles at any
 // moment, so the tiles in flight together share a few row tiles and a few
 // column tiles: their operands stay in L2 across the group instead of being
-// streamed again from HBM for every row tile.
+// streamed again from HBM for every row tile. A group's row operands should
+// fit in kResidentBytes of L2; when 16 row tiles of a long K range do not
+// (the down projection and the gate/up input gradient at large f), the
+// group has 8, which also makes the 74 tiles in flight together nearly
+// square (fewest distinct operand blocks per wave). The weight gradient
+// keeps the whole d-side operand of an expert (xp for dWg / dWu, dyp for
+// dWd) in the group when it fits, so the long f-side operand (dh1, dh2, a)
+// streams through L2 once.
 constexpr int kRasterRows = 16;
 constexpr int kRasterM = 8;
+constexpr long long kResidentBytes = 48ll << 20;
 constexpr long long kWaitLimit = 2000000000LL;  // about one second of SM cycles
 constexpr uint32_t kTmemCols = 512;
 
@@ -118,6 +126,13 @@ struct Traits {
   static constexpr uint32_t B_BYTES = (PAIR ? BN / 2 : BN) * BK * 2;    // per CTA
   static constexpr uint32_t STAGE_TX = (A_BYTES + B_BYTES) * (PAIR ? 2 : 1);  // all CTAs
   static constexpr uint32_t IDESC = umma_idesc_bf16(TM, BN, A_MN, B_MN);
+  // Pair kinds whose tile columns run over f (dgrad down; dWg and dWu of the
+  // weight gradient): when f is not a multiple of BN, a last column tile with
+  // at most BN / 2 valid columns runs MMAs of half the width, each CTA staging
+  // the first 64 of its B columns from the tile's midpoint instead of
+  // BN / 2 past it.
+  static constexpr bool NARROW = PAIR && BN == 256 && (KIND == kBwdDgradDown || KIND == kWgrad);
+  static constexpr uint32_t IDESC_NARROW = umma_idesc_bf16(TM, BN / 2, A_MN, B_MN);
   // N extent of one output tile (gate/up: 128 f columns, each with its gate
   // and up accumulator, together the MMA's N = 256)
   static constexpr int NTILE = KIND == kFwdGateUp ? 128 : BN;
@@ -142,6 +157,7 @@ struct TileInfo {
   int m0;    // wgrad: first f index of the tile
   int n0;    // first output column of the tile
   int prod;  // wgrad: 0 dWg, 1 dWu, 2 dWd
+  int narrow;  // half-width MMAs (Traits::NARROW)
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -217,21 +233,27 @@ __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d,
     }
     const int mt = ti.prod < 2 ? ceil_div(d, Tr::TM) : ceil_div(f, Tr::TM);
     int mi, ni;
-    raster(rem, mt, nt, kRasterM, mi, ni);
+    if (2ll * d * cnt > kResidentBytes) raster(rem, mt, nt, kRasterM, mi, ni);
+    else if (ti.prod < 2) raster(rem, mt, nt, mt, mi, ni);  // M (over d) fastest
+    else raster(rem, nt, mt, nt, ni, mi);                    // N (over d) fastest
     ti.m0 = mi * Tr::TM;
     ti.n0 = ni * BN;
     ti.row0 = base;
     ti.rows = cnt;
+    ti.narrow = Tr::NARROW && ti.prod < 2 && f - ti.n0 <= BN / 2;
   } else {
     const int n_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? f : d;
     const int nt = ceil_div(n_extent, Tr::NTILE);
+    const int k_extent = (KIND == kFwdGateUp || KIND == kBwdDgradDown) ? d : (KIND == kFwdDown ? f : 2 * f);
+    const int g = 2ll * kRasterRows * Tr::TM * k_extent <= kResidentBytes ? kRasterRows : kRasterRows / 2;
     int mi, ni;
-    raster(local, ceil_div(cnt, Tr::TM), nt, kRasterRows, mi, ni);
+    raster(local, ceil_div(cnt, Tr::TM), nt, g, mi, ni);
     ti.n0 = ni * Tr::NTILE;
     ti.row0 = base + mi * Tr::TM;
     ti.rows = min(Tr::TM, cnt - mi * Tr::TM);
     ti.m0 = 0;
     ti.prod = 0;
+    ti.narrow = Tr::NARROW && f - ti.n0 <= BN / 2;
   }
   return ti;
 }
@@ -283,6 +305,7 @@ __device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& 
   const int k0 = kb * BK;
   const int arow = ti.row0 + BM * cta;
   constexpr int HALF = BN / 2;
+  const int bh = ti.narrow ? HALF / 2 : HALF;  // B columns of the even CTA
   if (KIND == kFwdGateUp) {
     if (load_a) tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
     tma_load_3d_pair(b_dst, cta == 0 ? &m.b0 : &m.b1, bar, k0, ti.n0, ti.e);
@@ -293,7 +316,7 @@ __device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& 
     tma_load_2d_pair(a_dst, &m.a0, bar, k0, arow);
 #pragma unroll
     for (int j = 0; j < HALF / 64; ++j)
-      tma_load_3d_pair(b_dst + j * 8192, &m.b0, bar, ti.n0 + HALF * cta + 64 * j, k0, ti.e);
+      tma_load_3d_pair(b_dst + j * 8192, &m.b0, bar, ti.n0 + bh * cta + 64 * j, k0, ti.e);
   } else if (KIND == kBwdDgradGateUp) {
     const int half = ceil_div(f, BK);
     const bool second = kb >= half;
@@ -313,7 +336,7 @@ __device__ __forceinline__ void issue_loads_pair(const Maps& m, const TileInfo& 
     }
 #pragma unroll
     for (int j = 0; j < HALF / 64; ++j)
-      tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + HALF * cta + 64 * j, r);
+      tma_load_2d_pair(b_dst + j * 8192, bm, bar, ti.n0 + bh * cta + 64 * j, r);
   }
 }
 
@@ -646,13 +669,13 @@ __device__ __forceinline__ bool epilogue_swiglu_bwd(const Params& p, const Maps&
 // One K16 step of a stage: MMA of the stage's A and B at K offset 16 * kk.
 template <typename Tr, bool PAIR>
 __device__ __forceinline__ void issue_mma(uint32_t dtm, uint32_t a_addr, uint32_t b_addr, int kk,
-                                          uint32_t accumulate) {
+                                          uint32_t idesc, uint32_t accumulate) {
   const uint64_t adesc = Tr::A_MN ? umma_desc_sw128(a_addr + kk * 2048, 8192, 1024)
                                   : umma_desc_sw128(a_addr + kk * 32, 16, 1024);
   const uint64_t bdesc = Tr::B_MN ? umma_desc_sw128(b_addr + kk * 2048, 8192, 1024)
                                   : umma_desc_sw128(b_addr + kk * 32, 16, 1024);
-  if (PAIR) mma_bf16_pair(dtm, adesc, bdesc, Tr::IDESC, accumulate);
-  else mma_bf16(dtm, adesc, bdesc, Tr::IDESC, accumulate);
+  if (PAIR) mma_bf16_pair(dtm, adesc, bdesc, idesc, accumulate);
+  else mma_bf16(dtm, adesc, bdesc, idesc, accumulate);
 }
 
 // The MMA issuer's wait for a stage: its TMA loads (and, in a gathered
@@ -870,6 +893,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, s_abort, kWaitLimit)) break;
       tc_fence_after();
       const uint32_t dtm = tmem_base + acc * BN;
+      const uint32_t idesc = ti.narrow ? Tr::IDESC_NARROW : Tr::IDESC;
       // Full 64-deep K blocks: four MMAs each as straight-line code (a loop
       // with a run-time bound, or a branch, between them leaves the tensor
       // pipe idle between instructions).
@@ -885,7 +909,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
           const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, (kb | kk) != 0 ? 1u : 0u);
+            issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, idesc, (kb | kk) != 0 ? 1u : 0u);
           // the stage is free in both CTAs once these MMAs have read it
           if (PAIR) mma_commit_pair_multicast(&empty[stage], 0x3);
           else mma_commit(&empty[stage]);
@@ -933,7 +957,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
             const uint32_t a_addr = smem_u32(sA + stage * Tr::A_BYTES);
             const uint32_t b_addr = smem_u32(sB + stage * Tr::B_BYTES);
             for (int kk = 0; kk < ksteps; ++kk)
-              issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, (kb | kk) != 0 ? 1u : 0u);
+              issue_mma<Tr, PAIR>(dtm, a_addr, b_addr, kk, idesc, (kb | kk) != 0 ? 1u : 0u);
             if (PAIR) mma_commit_pair_multicast(&empty[stage], 0x3);
             else mma_commit(&empty[stage]);
           }
