@@ -183,18 +183,22 @@ class ClockSampler:
 
 # ------------------------------------------------------------- CPU oracle
 
-def oracle_step_fn(w, params_np, x_np, dY_np):
+def oracle_step_fn(w, params_np, x_np, dY_np, aux_coef: float = 0.0):
     """One oracle pass over the first n tokens of a microbatch (a bounded
     sample): forward, and backward with every parameter gradient for a
-    forward+backward workload."""
+    forward+backward workload; with a balance-loss coefficient, the loss and
+    its metrics in the forward and its gradient in the backward."""
     import oracle
 
     def step(n: int):
         x = x_np[:n]
         P = params_np
         fw = oracle.layer_forward(x, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], w.k, w.ep_groups)
+        if aux_coef:
+            oracle.aux_loss(fw["z"], fw["counts"], w.k, aux_coef)
         if w.backward:
-            oracle.layer_backward(fw, x, dY_np[:n], P["Wr"], P["Wg"], P["Wu"], P["Wd"], w.k)
+            oracle.layer_backward(fw, x, dY_np[:n], P["Wr"], P["Wg"], P["Wu"], P["Wd"], w.k,
+                                  aux=(aux_coef, 1.0) if aux_coef else None)
     return step
 
 
@@ -231,20 +235,21 @@ def calibrate_sample(step, budget_s: float, T: int) -> int:
     return int(max(1, min(T, (budget_s - fixed) / per_token)))
 
 
-def _what(w) -> str:
-    return "fwd+bwd (all parameter gradients)" if w.backward else "fwd"
+def _what(w, aux_coef: float = 0.0) -> str:
+    what = "fwd+bwd (all parameter gradients)" if w.backward else "fwd"
+    return what + (f" with the balance loss (coefficient {aux_coef})" if aux_coef else "")
 
 
-def cpu_baseline(w, budget_s: float = 15.0):
+def cpu_baseline(w, budget_s: float = 15.0, aux_coef: float = 0.0):
     import oracle
     P, x, dY = oracle_inputs(w)
-    step = oracle_step_fn(w, P, x, dY)
+    step = oracle_step_fn(w, P, x, dY, aux_coef)
     n = calibrate_sample(step, budget_s, w.T[0])
     t0 = time.perf_counter()
     step(n)
     dt = time.perf_counter() - t0
     return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"oracle {_what(w)} of the first {n} of the {w.T[0]} tokens of the first "
+            "sample": f"oracle {_what(w, aux_coef)} of the first {n} of the {w.T[0]} tokens of the first "
                       f"microbatch ({dt:.1f} s of CPU work)"}
 
 
@@ -254,7 +259,7 @@ def run_reference(args, w):
         return 0
     import oracle
     P, x, dY = oracle_inputs(w)
-    step = oracle_step_fn(w, P, x, dY)
+    step = oracle_step_fn(w, P, x, dY, args.aux_loss)
     per_step_budget = max(0.5, 150.0 / max(1, args.steps + args.warmup))
     n = calibrate_sample(step, per_step_budget, w.T[0])
     for _ in range(args.warmup):
@@ -273,7 +278,7 @@ def run_reference(args, w):
         "gpus_used": 0, "ranks_working": 1,
         "config": dict(workload_config(w), parallelism=f"{args.parallel}{args.gpus}"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"each step: oracle {_what(w)} of the first {n} tokens of the first "
+                         "sample": f"each step: oracle {_what(w, args.aux_loss)} of the first {n} tokens of the first "
                                    f"microbatch"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -499,7 +504,7 @@ def time_layer(w, args, R, with_e2e: bool = True):
     batches = [workloads.make_batch(w, mb=mb, device=dev, seed=R.batch_seed) for mb in range(len(w.T))]
     fused = args.dispatch == "fused"
     layer = MoELayer(params, w.k, w.ep_groups, max_tokens=max(w.T), checkpoint=args.checkpoint,
-                     fused_dispatch=fused)
+                     fused_dispatch=fused, aux_coef=args.aux_loss)
     stream = torch.cuda.current_stream(dev)
     rec = Recorder(stream)
 
@@ -631,7 +636,9 @@ def run_native(args, w):
         "options": {"dispatch": ("fused: expert rows gathered from x inside the GEMM operand loads, "
                                  "no permuted copy" if sfx else "permute: rows copied to xp first"),
                     "activations": ("checkpointed: h1, h2 rebuilt in the backward" if args.checkpoint
-                                    else "stored")},
+                                    else "stored"),
+                    "balance_loss": (f"coefficient {args.aux_loss}: loss, importance and entropy in the "
+                                     "forward, its gradient in the backward" if args.aux_loss else "off")},
     }
     gemm_names = [n + s for n in GEMM_CALLS for s in ("", "_gather") if n + s in call_ms]
     if gemm_names:
@@ -689,7 +696,7 @@ def run_native(args, w):
         line["forward_only"] = {n: forward_line(workloads.WORKLOADS[n], args, R) for n in FORWARD_EXTRAS}
     if R.rank == 0 and R.world == 1 and not args.no_cpu_baseline:
         try:
-            line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget, aux_coef=args.aux_loss)
         except Exception as ex:  # report, do not hide
             line["cpu_baseline"] = {"error": repr(ex)}
     if R.prints:
@@ -796,6 +803,9 @@ def main(argv=None):
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the forward-only lines reported beside the headline workload")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--aux-loss", type=float, default=0.0,
+                    help="Switch-style balance-loss coefficient: the forward also computes the loss "
+                         "and the routing metrics, the backward adds its gradient (0: off)")
     ap.add_argument("--checkpoint", action="store_true",
                     help="activation checkpointing: h1, h2 rebuilt in the backward")
     ap.add_argument("--dispatch", choices=["permute", "fused"], default="permute",
@@ -804,6 +814,10 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.aux_loss < 0:
+        ap.error("--aux-loss must be non-negative")
+    if args.aux_loss and args.parallel == "ep":
+        ap.error("--aux-loss runs with the data-parallel layer (--parallel dp)")
     if args.gpus < 1:
         ap.error("--gpus must be at least 1")
     env_world = os.environ.get("WORLD_SIZE")

@@ -97,3 +97,21 @@ def test_gpus_must_match_the_launchers_world_size():
                    env_extra={"WORLD_SIZE": "1", "RANK": "0", "LOCAL_RANK": "0"})
     assert r.returncode != 0
     assert "WORLD_SIZE=1" in r.stderr
+
+
+def test_reference_arm_with_the_balance_loss():
+    """`--aux-loss` reaches the reference arm: its oracle step computes the
+    loss and adds its gradient, and the line says so."""
+    import json
+    r = _run_bench(["--impl", "reference", "--workload", "tiny_fp32", "--aux-loss", "0.01", "--steps", "3",
+                    "--warmup", "3"])
+    assert r.returncode == 0, r.stdout + r.stderr
+    line = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")][0]
+    assert "balance loss (coefficient 0.01)" in line["cpu_baseline"]["sample"]
+    assert line["value"] > 0
+
+
+def test_balance_loss_needs_the_data_parallel_layer():
+    r = _run_bench(["--aux-loss", "0.01", "--parallel", "ep", "--workload", "tiny_fp32"])
+    assert r.returncode != 0
+    assert "--parallel dp" in r.stderr

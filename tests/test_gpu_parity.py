@@ -118,6 +118,13 @@ LAYER_CASES = [
     # largest), and top-32 (the largest k of the routing and combine kernels)
     ("bf16_max_experts", 600, 128, 1024, 8, 64, "bf16", 16, True),
     ("bf16_top32", 200, 128, 64, 32, 128, "bf16", 4, False),
+    # the GEMMs' tile orders for operands that do not fit in L2 beside each
+    # other: K ranges of the down projection (f) and of the input gradient
+    # (2f) too long for 16 row tiles of 256 rows (groups of 8, with 9 row
+    # tiles per expert), and an expert whose d-side operand (2 d rows bytes,
+    # 52 MB here) is too large to stay resident in the weight gradient
+    ("bf16_long_k_row_groups", 2200, 64, 2, 2, 6400, "bf16", 1, False),
+    ("bf16_wgrad_large_expert", 6300, 4096, 2, 1, 264, "bf16", 1, True),
     ("f32_tiny", 256, 64, 4, 2, 128, "f32", 2, True),
     ("f32_odd", 100, 48, 3, 2, 20, "f32", 1, False),
 ]
