@@ -212,53 +212,116 @@ cudaError_t launch_aux_loss_bwd(const float* z, const int32_t* counts, int64_t T
 }
 
 // ----------------------------------------------------- dense router backward
+//
+// The balance loss's logit gradient dz is dense over the experts, so its
+// router backward is two small dense products, dX += dz Wr ([T, E] x [E, d])
+// and dWr (+)= dz^T x ([E, T] x [T, d]) with db (+)= the column sums of dz,
+// on fp32 FFMA register tiles fed from operands staged as fp32 in shared
+// memory. Each output is summed in a fixed order (e ascending for dX; tokens
+// ascending inside 256-token chunks, then the chunks in order, for dWr), so
+// the result does not depend on scheduling. Experts are staged EC at a time
+// (16 when E <= 16, else 32), so no FMA runs on padding experts beyond the
+// last chunk's. A thread's 8 columns are two groups of 4, c0 + 4 tx and
+// c0 + 64 + 4 tx, so each quarter-warp's 16-byte shared loads cover 128
+// contiguous bytes.
 
-constexpr int kDenseTile = 64;   // tokens (dX) or experts (dWr) x 64 columns per block
-constexpr int kDenseChunk = 256; // tokens per dWr partial
+constexpr int kDenseTokens = 64;   // tokens per dX block and per dWr staging step
+constexpr int kDenseCols = 128;    // columns per block
+constexpr int kDenseChunk = 256;   // tokens per dWr partial
 
 int dense_router_chunks(int64_t T) {
   return static_cast<int>((T + kDenseChunk - 1) / kDenseChunk);
 }
 
-// dX[t, i] += sum_e dz[t,e] Wr[e,i]. Block: 64 tokens x 64 columns, 128
-// threads, each 8 tokens x 4 columns; e in chunks of 64 staged as fp32.
-template <typename T>
+// Elements i .. i + 3 of a row as floats, zero at or past n. VEC: one 8-byte
+// (bf16) or 16-byte (fp32) load; the row start and i are multiples of 4
+// elements and the base is aligned to 4 elements (checked at launch).
+template <typename T, bool VEC>
+__device__ __forceinline__ float4 load4(const T* row, int i, int n) {
+  if (VEC && i + 4 <= n) {
+    if constexpr (sizeof(T) == 2) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(row + i));
+      const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+      const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+      return make_float4(lo.x, lo.y, hi.x, hi.y);
+    } else {
+      return __ldg(reinterpret_cast<const float4*>(row + i));
+    }
+  }
+  float v[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) v[q] = i + q < n ? to_f32(row[i + q]) : 0.0f;
+  return make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// row[i + q] = row[i + q] + a[q] (one rounding to T) for q < 4, i + q < n.
+template <typename T, bool VEC>
+__device__ __forceinline__ void add4(T* row, int i, int n, const float (&a)[4]) {
+  if (VEC && i + 4 <= n) {
+    if constexpr (sizeof(T) == 2) {
+      uint2* p = reinterpret_cast<uint2*>(row + i);
+      uint2 u = *p;
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+      const float2 lo = __bfloat1622float2(h[0]), hi = __bfloat1622float2(h[1]);
+      h[0] = __floats2bfloat162_rn(lo.x + a[0], lo.y + a[1]);
+      h[1] = __floats2bfloat162_rn(hi.x + a[2], hi.y + a[3]);
+      *p = u;
+    } else {
+      float4* p = reinterpret_cast<float4*>(row + i);
+      float4 u = *p;
+      u.x += a[0]; u.y += a[1]; u.z += a[2]; u.w += a[3];
+      *p = u;
+    }
+    return;
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (i + q < n) row[i + q] = from_f32<T>(to_f32(row[i + q]) + a[q]);
+}
+
+// dX[t, i] += sum_e dz[t,e] Wr[e,i]. Block: 64 tokens x 128 columns, 128
+// threads, each 8 tokens x 8 columns.
+template <typename T, int EC, bool VEC>
 __global__ void __launch_bounds__(128) dense_dx_kernel(const float* __restrict__ dz,
                                                        const T* __restrict__ Wr, int64_t Ttok,
                                                        int d, int E, T* __restrict__ dX) {
-  __shared__ __align__(16) float s_dz[kDenseTile][kDenseTile + 4];  // [e][token]
-  __shared__ __align__(16) float s_w[kDenseTile][kDenseTile + 4];   // [e][column]
+  __shared__ __align__(16) float s_dz[EC][kDenseTokens + 4];  // [e][token]
+  __shared__ __align__(16) float s_w[EC][kDenseCols + 4];     // [e][column]
   const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;  // columns tx*4.., tokens ty*8..
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDenseTile;
-  const int i0 = blockIdx.y * kDenseTile;
-  float acc[8][4];
+  const int tx = tid % 16, ty = tid / 16;  // columns 4 tx, 64 + 4 tx; tokens 8 ty ..
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kDenseTokens;
+  const int i0 = blockIdx.y * kDenseCols;
+  float acc[8][8];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
-  for (int e0 = 0; e0 < E; e0 += kDenseTile) {
-    for (int idx = tid; idx < kDenseTile * kDenseTile; idx += 128) {
-      const int tt = idx / kDenseTile, ee = idx % kDenseTile;  // consecutive threads: consecutive e
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.0f;
+  for (int e0 = 0; e0 < E; e0 += EC) {
+    for (int idx = tid; idx < kDenseTokens * EC; idx += 128) {
+      const int tt = idx / EC, ee = idx % EC;  // consecutive threads: consecutive e
       const int64_t t = t0 + tt;
       const int e = e0 + ee;
       s_dz[ee][tt] = (t < Ttok && e < E) ? dz[t * E + e] : 0.0f;
-      const int ew = e0 + idx / kDenseTile, iw = i0 + idx % kDenseTile;
-      s_w[idx / kDenseTile][idx % kDenseTile] =
-          (ew < E && iw < d) ? to_f32(Wr[static_cast<int64_t>(ew) * d + iw]) : 0.0f;
+    }
+    for (int idx = tid; idx < EC * (kDenseCols / 4); idx += 128) {
+      const int ee = idx / (kDenseCols / 4), c4 = 4 * (idx % (kDenseCols / 4));
+      const int e = e0 + ee;
+      *reinterpret_cast<float4*>(&s_w[ee][c4]) =
+          e < E ? load4<T, VEC>(Wr + static_cast<int64_t>(e) * d, i0 + c4, d) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    const int ee_end = min(kDenseTile, E - e0);
+    const int ee_end = min(EC, E - e0);
     for (int ee = 0; ee < ee_end; ++ee) {
       const float4 za = *reinterpret_cast<const float4*>(&s_dz[ee][ty * 8]);
       const float4 zb = *reinterpret_cast<const float4*>(&s_dz[ee][ty * 8 + 4]);
-      const float4 w4 = *reinterpret_cast<const float4*>(&s_w[ee][tx * 4]);
+      const float4 wa = *reinterpret_cast<const float4*>(&s_w[ee][tx * 4]);
+      const float4 wb = *reinterpret_cast<const float4*>(&s_w[ee][64 + tx * 4]);
       const float zv[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-      const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+      const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
       for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = __fmaf_rn(zv[a], wv[c], acc[a][c]);
+        for (int c = 0; c < 8; ++c) acc[a][c] = __fmaf_rn(zv[a], wv[c], acc[a][c]);
     }
     __syncthreads();
   }
@@ -266,77 +329,93 @@ __global__ void __launch_bounds__(128) dense_dx_kernel(const float* __restrict__
   for (int a = 0; a < 8; ++a) {
     const int64_t t = t0 + ty * 8 + a;
     if (t >= Ttok) continue;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = i0 + tx * 4 + c;
-      if (i < d) {
-        T* p = dX + t * d + i;
-        *p = from_f32<T>(to_f32(*p) + acc[a][c]);
-      }
-    }
+    T* row = dX + t * d;
+    const float lo[4] = {acc[a][0], acc[a][1], acc[a][2], acc[a][3]};
+    const float hi[4] = {acc[a][4], acc[a][5], acc[a][6], acc[a][7]};
+    add4<T, VEC>(row, i0 + tx * 4, d, lo);
+    add4<T, VEC>(row, i0 + 64 + tx * 4, d, hi);
   }
 }
 
 // partial[chunk][e][i] = sum_{t in chunk} dz[t,e] x[t,i] and, for the first
 // column tile, partial_db[chunk][e] = sum_{t in chunk} dz[t,e]. Block: one
-// 256-token chunk x 64 experts x 64 columns, 128 threads, each 8 experts x 4
-// columns; tokens in steps of 64 staged as fp32, summed in token order.
-template <typename T>
+// 256-token chunk x EC experts x 128 columns, 128 threads, each EC / 8
+// experts x 8 columns; tokens in steps of 64, summed in token order.
+template <typename T, int EC, bool VEC>
 __global__ void __launch_bounds__(128) dense_dwr_partial_kernel(const T* __restrict__ x,
                                                                 const float* __restrict__ dz,
                                                                 int64_t Ttok, int d, int E,
                                                                 float* __restrict__ partial,
                                                                 float* __restrict__ partial_db) {
-  __shared__ __align__(16) float s_dz[kDenseTile][kDenseTile + 4];  // [token][e]
-  __shared__ __align__(16) float s_x[kDenseTile][kDenseTile + 4];   // [token][column]
+  constexpr int RE = EC / 8;
+  __shared__ __align__(16) float s_dz[kDenseTokens][EC + 4];       // [token][e]
+  __shared__ __align__(16) float s_x[kDenseTokens][kDenseCols + 4];  // [token][column]
   const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;  // columns tx*4.., experts ty*8..
+  const int tx = tid % 16, ty = tid / 16;  // columns 4 tx, 64 + 4 tx; experts RE ty ..
   const int chunk = blockIdx.x;
-  const int i0 = blockIdx.y * kDenseTile;
-  const int e0 = blockIdx.z * kDenseTile;
-  float acc[8][4];
-  float accb[8];
+  const int i0 = blockIdx.y * kDenseCols;
+  const int e0 = blockIdx.z * EC;
+  float acc[RE][8];
+  float accb[RE];
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
+  for (int a = 0; a < RE; ++a) {
     accb[a] = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) acc[a][c] = 0.0f;
+    for (int c = 0; c < 8; ++c) acc[a][c] = 0.0f;
   }
   const int64_t tbeg = static_cast<int64_t>(chunk) * kDenseChunk;
-  for (int64_t ts = tbeg; ts < tbeg + kDenseChunk && ts < Ttok; ts += kDenseTile) {
-    for (int idx = tid; idx < kDenseTile * kDenseTile; idx += 128) {
-      const int tt = idx / kDenseTile, cc = idx % kDenseTile;
+  const int64_t tend = min(tbeg + kDenseChunk, Ttok);
+  for (int64_t ts = tbeg; ts < tend; ts += kDenseTokens) {
+    for (int idx = tid; idx < kDenseTokens * EC; idx += 128) {
+      const int tt = idx / EC, ee = idx % EC;
       const int64_t t = ts + tt;
-      const int e = e0 + cc, i = i0 + cc;
-      const bool tok = t < Ttok && t < tbeg + kDenseChunk;
-      s_dz[tt][cc] = (tok && e < E) ? dz[t * E + e] : 0.0f;
-      s_x[tt][cc] = (tok && i < d) ? to_f32(x[t * d + i]) : 0.0f;
+      const int e = e0 + ee;
+      s_dz[tt][ee] = (t < tend && e < E) ? dz[t * E + e] : 0.0f;
+    }
+    for (int idx = tid; idx < kDenseTokens * (kDenseCols / 4); idx += 128) {
+      const int tt = idx / (kDenseCols / 4), c4 = 4 * (idx % (kDenseCols / 4));
+      const int64_t t = ts + tt;
+      *reinterpret_cast<float4*>(&s_x[tt][c4]) =
+          t < tend ? load4<T, VEC>(x + t * d, i0 + c4, d) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
-    for (int tt = 0; tt < kDenseTile; ++tt) {
-      const float4 za = *reinterpret_cast<const float4*>(&s_dz[tt][ty * 8]);
-      const float4 zb = *reinterpret_cast<const float4*>(&s_dz[tt][ty * 8 + 4]);
-      const float4 x4 = *reinterpret_cast<const float4*>(&s_x[tt][tx * 4]);
-      const float zv[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-      const float xv[4] = {x4.x, x4.y, x4.z, x4.w};
+    for (int tt = 0; tt < kDenseTokens; ++tt) {
+      float zv[RE];
+      if constexpr (RE == 4) {
+        const float4 z4 = *reinterpret_cast<const float4*>(&s_dz[tt][ty * 4]);
+        zv[0] = z4.x; zv[1] = z4.y; zv[2] = z4.z; zv[3] = z4.w;
+      } else {
 #pragma unroll
-      for (int a = 0; a < 8; ++a) {
+        for (int a = 0; a < RE; ++a) zv[a] = s_dz[tt][ty * RE + a];
+      }
+      const float4 xa = *reinterpret_cast<const float4*>(&s_x[tt][tx * 4]);
+      const float4 xb = *reinterpret_cast<const float4*>(&s_x[tt][64 + tx * 4]);
+      const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+      for (int a = 0; a < RE; ++a) {
         accb[a] += zv[a];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][c] = __fmaf_rn(zv[a], xv[c], acc[a][c]);
+        for (int c = 0; c < 8; ++c) acc[a][c] = __fmaf_rn(zv[a], xv[c], acc[a][c]);
       }
     }
     __syncthreads();
   }
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int e = e0 + ty * 8 + a;
+  for (int a = 0; a < RE; ++a) {
+    const int e = e0 + ty * RE + a;
     if (e >= E) continue;
     float* prow = partial + (static_cast<int64_t>(chunk) * E + e) * d;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int i = i0 + tx * 4 + c;
-      if (i < d) prow[i] = acc[a][c];
+    for (int h = 0; h < 2; ++h) {
+      const int i = i0 + 64 * h + tx * 4;
+      if (i + 4 <= d) {
+        *reinterpret_cast<float4*>(prow + i) =
+            make_float4(acc[a][4 * h], acc[a][4 * h + 1], acc[a][4 * h + 2], acc[a][4 * h + 3]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (i + q < d) prow[i + q] = acc[a][4 * h + q];
+      }
     }
     if (blockIdx.y == 0 && tx == 0) partial_db[static_cast<int64_t>(chunk) * E + e] = accb[a];
   }
@@ -366,23 +445,40 @@ __global__ void __launch_bounds__(256) dense_dwr_reduce_kernel(const float* __re
   }
 }
 
+template <typename T, int EC, bool VEC>
+static cudaError_t launch_dense_e(const T* x, const T* Wr, const float* dz, int64_t Ttok, int d,
+                                  int E, T* dX, float* partial, float* partial_db, cudaStream_t s) {
+  const unsigned gy = static_cast<unsigned>((d + kDenseCols - 1) / kDenseCols);
+  if (dX) {
+    dense_dx_kernel<T, EC, VEC><<<dim3(static_cast<unsigned>((Ttok + kDenseTokens - 1) / kDenseTokens), gy),
+                                  128, 0, s>>>(dz, Wr, Ttok, d, E, dX);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  dense_dwr_partial_kernel<T, EC, VEC><<<dim3(static_cast<unsigned>(dense_router_chunks(Ttok)), gy,
+                                              static_cast<unsigned>((E + EC - 1) / EC)),
+                                         128, 0, s>>>(x, dz, Ttok, d, E, partial, partial_db);
+  return cudaGetLastError();
+}
+
 template <typename T>
 static cudaError_t launch_dense_t(const T* x, const T* Wr, const float* dz, int64_t Ttok, int d,
                                   int E, T* dX, float* dWr, float* db, int accumulate,
                                   float* partial, cudaStream_t s) {
-  const unsigned gy = static_cast<unsigned>((d + kDenseTile - 1) / kDenseTile);
-  if (dX) {
-    dense_dx_kernel<T><<<dim3(static_cast<unsigned>((Ttok + kDenseTile - 1) / kDenseTile), gy), 128,
-                         0, s>>>(dz, Wr, Ttok, d, E, dX);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   const int nchunk = dense_router_chunks(Ttok);
   float* partial_db = partial + static_cast<int64_t>(nchunk) * E * d;
-  dense_dwr_partial_kernel<T><<<dim3(static_cast<unsigned>(nchunk), gy,
-                                     static_cast<unsigned>((E + kDenseTile - 1) / kDenseTile)),
-                                128, 0, s>>>(x, dz, Ttok, d, E, partial, partial_db);
-  cudaError_t e = cudaGetLastError();
+  // vector accesses of 4 elements need every row start aligned to them (d is
+  // a multiple of 4) and so the base pointers
+  const uintptr_t al = 4 * sizeof(T) - 1;
+  const bool vec = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(Wr) |
+                     reinterpret_cast<uintptr_t>(dX)) & al) == 0;
+  cudaError_t e;
+  if (E <= 16)
+    e = vec ? launch_dense_e<T, 16, true>(x, Wr, dz, Ttok, d, E, dX, partial, partial_db, s)
+            : launch_dense_e<T, 16, false>(x, Wr, dz, Ttok, d, E, dX, partial, partial_db, s);
+  else
+    e = vec ? launch_dense_e<T, 32, true>(x, Wr, dz, Ttok, d, E, dX, partial, partial_db, s)
+            : launch_dense_e<T, 32, false>(x, Wr, dz, Ttok, d, E, dX, partial, partial_db, s);
   if (e != cudaSuccess) return e;
   const int64_t n = static_cast<int64_t>(E) * d + E;
   const unsigned blocks = static_cast<unsigned>((n + 255) / 256 < 148 * 8 ? (n + 255) / 256 : 148 * 8);

@@ -50,14 +50,31 @@ def test_aux_loss_of_an_empty_batch_is_zero():
         assert not t.any(), n
 
 
-@pytest.mark.parametrize("dtype,T,d,E", [("bf16", 700, 192, 70), ("f32", 333, 200, 9), ("bf16", 64, 64, 64)])
-def test_dense_router_backward_matches_oracle(dtype, T, d, E):
+def _offset_copy(t, offset):
+    """A copy of t whose data starts `offset` elements into a fresh buffer
+    (offset 2: 4 or 8 bytes past an aligned start, so the kernels take their
+    element-by-element path)."""
+    if not offset:
+        return t.contiguous()
+    buf = torch.empty(t.numel() + offset, dtype=t.dtype, device=t.device)
+    v = buf[offset:].view(t.shape)
+    v.copy_(t)
+    return v
+
+
+# E <= 16 (experts staged 16 at a time) and above (32 at a time, a partial
+# last chunk at E = 70); d with a partial 128-column tile; T off the 64-token
+# steps and 256-token chunks; aligned and misaligned operands
+@pytest.mark.parametrize("dtype,T,d,E,offset", [("bf16", 700, 192, 70, 0), ("f32", 333, 200, 9, 0),
+                                                ("bf16", 64, 64, 64, 0), ("bf16", 1000, 256, 16, 0),
+                                                ("bf16", 300, 136, 40, 2), ("f32", 130, 68, 5, 2)])
+def test_dense_router_backward_matches_oracle(dtype, T, d, E, offset):
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     g = torch.Generator(device="cpu").manual_seed(T * 31 + E)
-    x = torch.randn((T, d), generator=g).to(tdt).to(DEV)
-    Wr = (torch.randn((E, d), generator=g) * 0.05).to(tdt).to(DEV)
+    x = _offset_copy(torch.randn((T, d), generator=g).to(tdt).to(DEV), offset)
+    Wr = _offset_copy((torch.randn((E, d), generator=g) * 0.05).to(tdt).to(DEV), offset)
     dz = (torch.randn((T, E), generator=g) * 0.1).to(DEV)
-    dX = torch.randn((T, d), generator=g).to(tdt).to(DEV)
+    dX = _offset_copy(torch.randn((T, d), generator=g).to(tdt).to(DEV), offset)
     dWr = torch.randn((E, d), generator=g).to(DEV)
     db = torch.randn(E, generator=g).to(DEV)
     dX0, dWr0, db0 = (to_np(t).astype(np.float64) for t in (dX, dWr, db))
