@@ -118,11 +118,27 @@ __global__ void __launch_bounds__(NT) router_logits_kernel(const T* __restrict__
         for (int c = 0; c < RE; ++c) wv[c] = ws[ii][logit_pad(tx * RE + c)];
       }
     };
+    // with two experts per thread (E <= 16), both chains of a token in one
+    // packed instruction (__ffma2_rn rounds each component as __fmaf_rn
+    // does, so the chains are the same): 14-18% faster at d = 4096; with 8
+    // per thread the packed form measured 5-20% slower
     auto fma_step = [&](const float (&xv)[8], const float (&wv)[RE]) {
 #pragma unroll
-      for (int a = 0; a < 8; ++a)
+      for (int a = 0; a < 8; ++a) {
+        if constexpr (RE == 2) {
+          const float2 xx = make_float2(xv[a], xv[a]);
 #pragma unroll
-        for (int c = 0; c < RE; ++c) acc[a][c] = __fmaf_rn(xv[a], wv[c], acc[a][c]);
+          for (int c = 0; c < RE; c += 2) {
+            const float2 r = __ffma2_rn(xx, make_float2(wv[c], wv[c + 1]),
+                                        make_float2(acc[a][c], acc[a][c + 1]));
+            acc[a][c] = r.x;
+            acc[a][c + 1] = r.y;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < RE; ++c) acc[a][c] = __fmaf_rn(xv[a], wv[c], acc[a][c]);
+        }
+      }
     };
     load_step(0, xa, wa);
     int ii = 0;
