@@ -83,7 +83,7 @@ def test_route_with_selected_minus_inf_is_a_defined_softmax():
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("T,d,E", [(1, 64, 4), (300, 264, 8), (129, 1024, 16), (1000, 512, 64),
                                    (77, 128, 100), (3, 4096, 16), (5000, 256, 16), (700, 136, 12),
-                                   (4096, 64, 1)])
+                                   (4096, 64, 1), (600, 200, 24), (2000, 128, 32), (500, 96, 40)])
 def test_router_logits_bitexact(dtype, T, d, E):
     """Bit-exact with the oracle's fixed-order fp32 logits on both kernels: one
     thread per logit for T E <= 4096, the 64-token tiles above it."""
