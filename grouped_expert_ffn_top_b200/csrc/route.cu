@@ -163,36 +163,78 @@ __global__ void __launch_bounds__(NT) router_logits_kernel(const T* __restrict__
   }
 }
 
-// Small batches (T E <= kLogitSmallOutputs): one thread per logit, the
-// fixed-order fma chain over i = 0..d-1 fed by 16-byte loads of its token's
-// x row and its expert's Wr row (four loads in flight). The tiled kernel
-// above stages 64-token tiles through shared memory chunk by chunk, which for
-// a handful of tokens is a chain of load latencies; here the chain is the
-// d dependent FMAs themselves. Same order of operations, same result bits.
+// Small batches (T E <= kLogitSmallOutputs): one warp per logit. The chain
+// of d dependent FMAs is the logit's time, so one lane runs it over the
+// token's x row and the expert's Wr row staged as fp32 in the warp's shared
+// memory, kSmallCols columns at a time; before each chunk's chain the warp
+// issues the 16-byte loads of the next chunk into registers, which land while
+// the chain runs, and stores them after it. Same order of operations as the
+// tiled kernel above, same result bits.
 constexpr int64_t kLogitSmallOutputs = 4096;
+constexpr int kSmallCols = 512;
+constexpr int kSmallWarps = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(128) router_logits_small_kernel(const T* __restrict__ x,
-                                                                  const T* __restrict__ Wr,
-                                                                  const float* __restrict__ b,
-                                                                  int64_t Ttok, int d, int E,
-                                                                  float* __restrict__ z) {
-  constexpr int VE = Vec16<T>::N;
-  const int64_t o = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (o >= Ttok * E) return;
+__global__ void __launch_bounds__(32 * kSmallWarps) router_logits_small_kernel(
+    const T* __restrict__ x, const T* __restrict__ Wr, const float* __restrict__ b, int64_t Ttok,
+    int d, int E, float* __restrict__ z) {
+  constexpr int VE = Vec16<T>::N;           // elements per 16-byte vector
+  constexpr int VPL = kSmallCols / VE / 32;  // vectors per lane per row and chunk
+  __shared__ __align__(16) float st[kSmallWarps][2][kSmallCols];  // [warp][x, Wr][column]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t o = static_cast<int64_t>(blockIdx.x) * kSmallWarps + warp;
+  if (o >= Ttok * E) return;  // whole warps only: no block-wide barrier below
   const int64_t t = o / E;
   const int e = static_cast<int>(o % E);
   const T* xr = x + t * d;
   const T* wr = Wr + static_cast<int64_t>(e) * d;
-  float acc = 0.0f;
-#pragma unroll 4
-  for (int i = 0; i < d; i += VE) {
-    const Vec16<T> xv = ld16(xr + i);
-    const Vec16<T> wv = ld16(wr + i);
+  Vec16<T> px[VPL], pw[VPL];
+  auto gload = [&](int i0) {
 #pragma unroll
-    for (int q = 0; q < VE; ++q) acc = __fmaf_rn(xv.get(q), wv.get(q), acc);
+    for (int j = 0; j < VPL; ++j) {
+      const int c = i0 + (lane + 32 * j) * VE;
+      if (c < d) {
+        px[j] = ld16(xr + c);
+        pw[j] = ld16(wr + c);
+      } else {
+        px[j].raw = pw[j].raw = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  };
+  auto sstore = [&]() {
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int c = (lane + 32 * j) * VE;
+#pragma unroll
+      for (int q = 0; q < VE; ++q) {
+        st[warp][0][c + q] = px[j].get(q);
+        st[warp][1][c + q] = pw[j].get(q);
+      }
+    }
+  };
+  float acc = 0.0f;
+  gload(0);
+  for (int i0 = 0; i0 < d; i0 += kSmallCols) {
+    sstore();
+    __syncwarp();
+    if (i0 + kSmallCols < d) gload(i0 + kSmallCols);
+    if (lane == 0) {
+      const float* xs = st[warp][0];
+      const float* ws = st[warp][1];
+      const int n = min(kSmallCols, d - i0);  // a multiple of 8 (d is)
+#pragma unroll 4
+      for (int i = 0; i < n; i += 4) {
+        const float4 xv = *reinterpret_cast<const float4*>(xs + i);
+        const float4 wv = *reinterpret_cast<const float4*>(ws + i);
+        acc = __fmaf_rn(xv.x, wv.x, acc);
+        acc = __fmaf_rn(xv.y, wv.y, acc);
+        acc = __fmaf_rn(xv.z, wv.z, acc);
+        acc = __fmaf_rn(xv.w, wv.w, acc);
+      }
+    }
+    __syncwarp();
   }
-  z[o] = __fadd_rn(acc, b ? b[e] : 0.0f);
+  if (lane == 0) z[o] = __fadd_rn(acc, b ? b[e] : 0.0f);
 }
 
 template <typename T>
@@ -200,8 +242,8 @@ static cudaError_t launch_router_logits_t(const T* x, const T* Wr, const float* 
                                           int d, int E, float* z, cudaStream_t s) {
   const unsigned gx = static_cast<unsigned>((Ttok + kLogitTokens - 1) / kLogitTokens);
   if (Ttok * E <= kLogitSmallOutputs) {
-    const unsigned blocks = static_cast<unsigned>((Ttok * E + 127) / 128);
-    router_logits_small_kernel<T><<<blocks, 128, 0, s>>>(x, Wr, b, Ttok, d, E, z);
+    const unsigned blocks = static_cast<unsigned>((Ttok * E + kSmallWarps - 1) / kSmallWarps);
+    router_logits_small_kernel<T><<<blocks, 32 * kSmallWarps, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 8) {
     router_logits_kernel<T, 8, 64><<<dim3(gx, 1), 64, 0, s>>>(x, Wr, b, Ttok, d, E, z);
   } else if (E <= 16) {
