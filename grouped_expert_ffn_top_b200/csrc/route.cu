@@ -118,10 +118,11 @@ __global__ void __launch_bounds__(NT) router_logits_kernel(const T* __restrict__
         for (int c = 0; c < RE; ++c) wv[c] = ws[ii][logit_pad(tx * RE + c)];
       }
     };
-    // with two experts per thread (E <= 16), both chains of a token in one
-    // packed instruction (__ffma2_rn rounds each component as __fmaf_rn
-    // does, so the chains are the same): 14-18% faster at d = 4096; with 8
-    // per thread the packed form measured 5-20% slower
+    // with two experts per thread (the tiles for E <= 16 and E <= 32), both
+    // chains of a token in one packed instruction (__ffma2_rn rounds each
+    // component as __fmaf_rn does, so the chains are the same): 14-18%
+    // faster at d = 4096, E = 16; with 8 per thread the packed form measured
+    // 5-20% slower
     auto fma_step = [&](const float (&xv)[8], const float (&wv)[RE]) {
 #pragma unroll
       for (int a = 0; a < 8; ++a) {
