@@ -201,11 +201,29 @@ struct Sched {
   const int* tstart;   // [E+1] first tile of each scheduled slot
   const int* order;    // [E] expert of each slot
   int E;
+  int total;  // tiles of the launch
+  int width;  // tiles in flight together (CTAs, or CTA pairs)
 };
+
+// Weight gradient: processing position g -> index in the tile list, whose
+// experts run longest first. Whole waves of `width` tiles alternate between
+// the front of the list (long K: MMA-bound) and its back (short K: bound by
+// the 256 KB fp32 store or add of each tile), and the last, partial wave
+// takes the middle remainder. Each CTA pair then alternates long and short
+// tiles, so a short tile's epilogue runs under a long tile's main loop
+// instead of the short tiles' epilogues running back to back at the end.
+__device__ __forceinline__ int interleave_waves(int g, int n, int width) {
+  const int waves = (n + width - 1) / width;
+  const int w = g / width, pos = g - w * width;
+  if (w == waves - 1) return (waves / 2) * width + pos;  // the middle remainder
+  if ((w & 1) == 0) return (w / 2) * width + pos;        // front chunk w / 2
+  return n - ((w - 1) / 2 + 1) * width + pos;            // back chunk (w - 1) / 2
+}
 
 template <int KIND, int BN, bool PAIR>
 __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d, int f) {
   using Tr = Traits<KIND, BN, PAIR>;
+  if (KIND == kWgrad) tile = interleave_waves(tile, s.total, s.width);
   int lo = 0, hi = s.E - 1;
   while (lo < hi) {  // largest slot whose first tile is <= tile
     const int mid = (lo + hi + 1) >> 1;
@@ -812,7 +830,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int total = *s_total;
-  const Sched sched{s_off, s_tstart, s_order, E};
+  const Sched sched{s_off, s_tstart, s_order, E, total, tile_step};
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
