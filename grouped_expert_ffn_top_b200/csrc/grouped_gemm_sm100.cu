@@ -59,6 +59,8 @@ constexpr int kMaxE = MOE_MAX_EXPERTS;
 constexpr int kRasterRows = 16;
 constexpr int kRasterM = 8;
 constexpr long long kResidentBytes = 48ll << 20;
+// weight gradient: experts with fewer rows have short-K tiles (interleave_waves)
+constexpr int kShortRows = 1024;
 constexpr long long kWaitLimit = 2000000000LL;  // about one second of SM cycles
 constexpr uint32_t kTmemCols = 512;
 
@@ -202,28 +204,33 @@ struct Sched {
   const int* order;    // [E] expert of each slot
   int E;
   int total;  // tiles of the launch
+  int nlong;  // weight gradient: tiles of the experts with at least kShortRows rows
   int width;  // tiles in flight together (CTAs, or CTA pairs)
 };
 
 // Weight gradient: processing position g -> index in the tile list, whose
-// experts run longest first. Whole waves of `width` tiles alternate between
-// the front of the list (long K: MMA-bound) and its back (short K: bound by
-// the 256 KB fp32 store or add of each tile), and the last, partial wave
-// takes the middle remainder. Each CTA pair then alternates long and short
-// tiles, so a short tile's epilogue runs under a long tile's main loop
-// instead of the short tiles' epilogues running back to back at the end.
-__device__ __forceinline__ int interleave_waves(int g, int n, int width) {
-  const int waves = (n + width - 1) / width;
-  const int w = g / width, pos = g - w * width;
-  if (w == waves - 1) return (waves / 2) * width + pos;  // the middle remainder
-  if ((w & 1) == 0) return (w / 2) * width + pos;        // front chunk w / 2
-  return n - ((w - 1) / 2 + 1) * width + pos;            // back chunk (w - 1) / 2
+// experts run longest first, so its first nlong tiles have a long K (MMA
+// bound) and the rest a short one (bound by the 256 KB fp32 store or add of
+// each tile). While both parts have a whole wave of `width` tiles left, waves
+// alternate between them, so each CTA pair alternates a long and a short tile
+// and the short tile's epilogue runs under the long tile's main loop; the
+// remaining tiles follow in list order. Experts of similar size are not
+// interleaved with each other, which would only mix their operands in L2.
+__device__ __forceinline__ int interleave_waves(int g, int n, int nlong, int width) {
+  const int m = min(nlong / width, (n - nlong) / width);  // alternating wave pairs
+  if (g < 2 * m * width) {
+    const int w = g / width, pos = g - w * width;
+    return (w & 1) ? nlong + (w >> 1) * width + pos : (w >> 1) * width + pos;
+  }
+  const int r = g - 2 * m * width;      // position among the rest
+  const int along = nlong - m * width;  // long tiles left
+  return r < along ? m * width + r : nlong + m * width + (r - along);
 }
 
 template <int KIND, int BN, bool PAIR>
 __device__ __forceinline__ TileInfo decode_tile(const Sched& s, int tile, int d, int f) {
   using Tr = Traits<KIND, BN, PAIR>;
-  if (KIND == kWgrad) tile = interleave_waves(tile, s.total, s.width);
+  if (KIND == kWgrad) tile = interleave_waves(tile, s.total, s.nlong, s.width);
   int lo = 0, hi = s.E - 1;
   while (lo < hi) {  // largest slot whose first tile is <= tile
     const int mid = (lo + hi + 1) >> 1;
@@ -733,6 +740,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(gfull + STAGES);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   int* s_total = const_cast<int*>(s_abort) + 1;
+  int* s_nlong = s_total + 1;
   int64_t* s_off = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(bars) + Tr::BAR_BYTES);
   int* s_tstart = reinterpret_cast<int*>(s_off + p.E + 1);
   int* s_order = s_tstart + p.E + 1;
@@ -818,9 +826,19 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
       if (s < E) s_tstart[s] = carry + inc - v;
       carry += __shfl_sync(0xffffffffu, inc, 31);
     }
+    __syncwarp();
     if (lane == 0) {
       s_tstart[E] = carry;
       *s_total = carry;
+      // slots run longest first: the long tiles end at the first short expert
+      int nlong = carry;
+      if (KIND == kWgrad)
+        for (int s = 0; s < E; ++s)
+          if (s_off[s_order[s] + 1] - s_off[s_order[s]] < kShortRows) {
+            nlong = s_tstart[s];
+            break;
+          }
+      *s_nlong = nlong;
     }
   }
   tc_fence_before();
@@ -830,7 +848,7 @@ __global__ void __launch_bounds__(Roles<KIND>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   const int total = *s_total;
-  const Sched sched{s_off, s_tstart, s_order, E, total, tile_step};
+  const Sched sched{s_off, s_tstart, s_order, E, total, *s_nlong, tile_step};
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
