@@ -260,6 +260,40 @@ def test_all_tokens_on_one_expert():
         assert_close_per(n, layer.grads[n], bw[n], 2e-2)
 
 
+@pytest.mark.parametrize("accumulate", [True, False])
+def test_weight_gradient_of_long_and_short_experts(accumulate):
+    """Seven experts with more than 1024 rows and seven with a few dozen, 12
+    weight-gradient tiles each: more than a wave (74 CTA pairs) of long tiles
+    and of short ones, so their waves alternate before the rest follows in
+    list order. Full dW per expert against the oracle, added to a non-zero
+    buffer or written over one."""
+    T, d, E, k, f = 4608, 512, 14, 2, 512
+    w = workloads.custom("long_short", T, d, E, k, f, dtype="bf16", bias="zero")
+    p = workloads.make_params(w, device=DEV, seed=0)
+    p["b"][:] = 0.0
+    p["b"][7:] = -1.0
+    bt = workloads.make_batch(w, device=DEV, seed=0)
+    layer = MoELayer(p, k, 1, max_tokens=T)
+    g0 = {n: torch.randn(layer.grads[n].shape, generator=torch.Generator().manual_seed(3)).to(DEV)
+          for n in ("dWg", "dWu", "dWd")}
+    for n in g0:
+        layer.grads[n].copy_(g0[n])
+    layer.forward(bt["x"])
+    layer.backward(bt["dY"], accumulate=accumulate)
+    torch.cuda.synchronize()
+    assert layer.device_errors() == 0
+    counts = to_np(layer.r["counts"])
+    assert (counts[:7] > 1024).all() and ((counts[7:] > 0) & (counts[7:] < 1024)).all(), counts
+    P = _np_params(p)
+    x64 = to_np(bt["x"]).astype(np.float64)
+    fw = oracle.layer_forward(x64, P["Wr"], P["b"], P["Wg"], P["Wu"], P["Wd"], k)
+    acc = {n: to_np(g0[n]).astype(np.float64) for n in g0} if accumulate else None
+    bw = oracle.layer_backward(fw, x64, to_np(bt["dY"]).astype(np.float64), P["Wr"], P["Wg"], P["Wu"],
+                               P["Wd"], k, acc=acc)
+    for n in ("dWg", "dWu", "dWd"):
+        assert_close_per(n, layer.grads[n], bw[n], TOL[torch.bfloat16])
+
+
 def test_long_ragged_weight_gradient_is_exact_and_reproducible():
     """Two experts of 4500 rows each: every weight-gradient tile runs 70 full
     64-row K blocks and a tail of 20 rows, ragged inside a 16-row MMA step.
