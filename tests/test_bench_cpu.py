@@ -115,3 +115,22 @@ def test_balance_loss_needs_the_data_parallel_layer():
     r = _run_bench(["--aux-loss", "0.01", "--parallel", "ep", "--workload", "tiny_fp32"])
     assert r.returncode != 0
     assert "--parallel dp" in r.stderr
+
+
+def test_roofline_traffic_is_reported_only_for_the_kernel_it_was_taken_on(monkeypatch):
+    """The committed DRAM bytes of the weight-gradient kernel are used while
+    the grouped GEMM source hashes as it did at capture time, and dropped
+    (None) once it changes."""
+    import json
+    import os
+    with open(os.path.join(bench.ROOT, "profiles", "ncu_traffic.json")) as fh:
+        t = json.load(fh)
+    for name, ent in t.items():
+        e = ent["grouped_ffn_wgrad"]
+        assert e["bytes_per_launch"] == int(round((e["dram_bytes_read_captured"] +
+                                                   e["dram_bytes_write_captured"]) * e["scale"]))
+        monkeypatch.setattr(bench, "source_hash", lambda h=e["source_hash"]: h)
+        assert bench.ncu_traffic("grouped_ffn_wgrad", name) == float(e["bytes_per_launch"])
+        monkeypatch.setattr(bench, "source_hash", lambda: "another kernel")
+        assert bench.ncu_traffic("grouped_ffn_wgrad", name) is None
+    assert bench.ncu_traffic("grouped_ffn_wgrad", "no such workload") is None
