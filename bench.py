@@ -107,10 +107,39 @@ GEMM_CALLS = ("grouped_ffn_fwd", "grouped_ffn_recompute", "grouped_ffn_dgrad", "
 MEM_CALLS = ("permute", "unpermute_combine", "unpermute_combine_bwd", "permute_bwd")
 
 
+def _code_only(src: str) -> str:
+    """C++ source without its comments and blank lines (string literals kept)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"':  # string literal, copied as is
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln.strip())
+
+
 def source_hash() -> str:
+    """Hash of the grouped GEMM's code (the kernel file and the headers it
+    builds on, comments and blank lines left out): the committed DRAM
+    counters of the kernel are used only while it matches."""
     h = hashlib.sha256()
-    with open(os.path.join(ROOT, "grouped_expert_ffn_top_b200", "csrc", "grouped_gemm_sm100.cu"), "rb") as fh:
-        h.update(fh.read())
+    csrc = os.path.join(ROOT, "grouped_expert_ffn_top_b200", "csrc")
+    for name in ("grouped_gemm_sm100.cu", "sm100.cuh", "common.cuh"):
+        with open(os.path.join(csrc, name), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

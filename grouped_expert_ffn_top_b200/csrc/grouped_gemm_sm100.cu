@@ -1,8 +1,9 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (sm_100a):
 // tcgen05.mma with fp32 accumulators in TMEM, operands staged by TMA into
-// 128-byte-swizzled shared memory, one persistent CTA per SM walking a tile
-// list built on the device from the expert offsets (no host synchronisation;
-// an expert with no rows contributes no tile).
+// 128-byte-swizzled shared memory, one persistent CTA pair (a cluster of two
+// SMs sharing each MMA) per two SMs walking a tile list built on the device
+// from the expert offsets (no host synchronisation; an expert with no rows
+// contributes no tile, except zero tiles of a weight gradient it writes).
 // (Grouped expert compute / grouped-GEMM: leap-finetune PR #26 Summary; ART
 // issue #917 Related.)
 //
@@ -12,18 +13,19 @@
 //   kBwdDgradDown   da = dyp Wd_e, epilogue dh1 = da h2 silu'(h1), dh2 = da silu(h1)
 //   kBwdDgradGateUp dxp = [dh1 | dh2] [Wg_e ; Wu_e]          (K = 2f)
 //   kWgrad          dWg_e^T += xp^T dh1, dWu_e^T += xp^T dh2, dWd_e^T += a^T dyp
-// The first four have a ragged M (the expert's rows, tiles of 128; rows of a
-// tile past the expert's end are computed and discarded). kWgrad has a ragged
-// K (the expert's rows): in the last K block the rows past the expert's end
-// are zeroed in shared memory before the MMA reads them.
+// The first four have a ragged M (the expert's rows, tiles of 256 = 128 per
+// CTA of the pair; rows of a tile past the expert's end are computed and
+// discarded). kWgrad has a ragged K (the expert's rows): in the last K block
+// the rows past the expert's end are zeroed in shared memory before the MMA
+// reads them.
 //
 // Warp roles: warp 0 issues TMA loads, warp 1 allocates TMEM and issues
-// tcgen05.mma (one lane), the remaining warps run the epilogue, each on its
-// TMEM lane quarter (warp % 4). The backward kinds, whose epilogues move the
-// most memory (SwiGLU backward, fp32 weight-gradient reductions), use eight
-// epilogue warps: two per lane quarter, one per half of the tile's columns.
-// Two TMEM accumulators let the epilogue of one tile overlap the main loop
-// of the next.
+// tcgen05.mma (one lane of the even CTA), the remaining warps run the
+// epilogue, each on its TMEM lane quarter (warp % 4). The weight gradient,
+// whose fp32 stores or reductions move the most memory, uses eight epilogue
+// warps: two per lane quarter, one per half of the tile's columns. Two TMEM
+// accumulators let the epilogue of one tile overlap the main loop of the
+// next.
 #include <cuda.h>
 
 #include "common.cuh"

@@ -134,3 +134,10 @@ def test_roofline_traffic_is_reported_only_for_the_kernel_it_was_taken_on(monkey
         monkeypatch.setattr(bench, "source_hash", lambda: "another kernel")
         assert bench.ncu_traffic("grouped_ffn_wgrad", name) is None
     assert bench.ncu_traffic("grouped_ffn_wgrad", "no such workload") is None
+
+
+def test_kernel_hash_ignores_comments_but_not_code():
+    code = 'asm volatile("tcgen05.commit // kept");  // the comment\n/* block */ int x = 1;\n\n'
+    assert bench._code_only(code) == 'asm volatile("tcgen05.commit // kept");\n int x = 1;'
+    assert bench._code_only(code.replace("the comment", "another one")) == bench._code_only(code)
+    assert bench._code_only(code.replace("x = 1", "x = 2")) != bench._code_only(code)
